@@ -1,0 +1,203 @@
+/*
+ * orthrus.h -- C ABI of the B200 (sm_100a) hot path of the Orthrus dual-view
+ * decode step.
+ *
+ * Method sources (web pages about "Orthrus: Memory-Efficient Parallel Token
+ * Generation via Dual-View Diffusion", arXiv 2605.12825):
+ *   [GIST]  gist.science summary, "Technische samenvatting": 2.1 dual-view
+ *           attention over one shared KV cache, 2.2 block mask M_diff
+ *           (causal context + bidirectional block), 2.3 inference consensus
+ *           (item 1 parallel projection of anchor + K-1 masks, item 2 AR check
+ *           of all K positions in one pass, item 3 longest greedy-matching
+ *           prefix, correction token, cache shortening).
+ *   [HN]    Hacker News thread "Orthrus-Qwen3: up to 7.8x tokens/forward on
+ *           Qwen3, identical output distribution", post #21 (K = 32, shared
+ *           KV cache, AR head accepts the longest matching prefix).
+ *   [ABS]   the paper's abstract: shared KV cache, exact consensus, O(1)
+ *           memory overhead.
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise, row-major
+ *     and densely packed.  bf16 means IEEE bfloat16 bits.  The caller owns
+ *     every buffer, including workspaces; the library allocates no device
+ *     memory.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default
+ *     stream.  Every call is asynchronous on `stream` and never synchronises.
+ *   - Return value: ORTHRUS_OK (0) or a negative orthrus_status.  Host-side
+ *     validation happens before any launch; on an error nothing is launched
+ *     and no output is touched.  ORTHRUS_ECUDA reports a launch failure.
+ *   - Conditions only the device can see (a committed length that would pass
+ *     the cache capacity, an accept length out of range) never trap: the
+ *     kernel clamps and, if `dev_status` is non-NULL, stores the first error
+ *     code there (atomically, only if it is still 0).  Callers zero it first.
+ *   - Waits inside kernels are bounded; a wait that gives up stores
+ *     ORTHRUS_ETIMEOUT in dev_status (when given) and the kernel returns.
+ *   - The library is built for sm_100a only.
+ */
+#ifndef ORTHRUS_H_
+#define ORTHRUS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ORTHRUS_OK = 0,
+  ORTHRUS_EINVAL = -1,       /* bad argument value (NULL pointer, K out of range, ...) */
+  ORTHRUS_ESHAPE = -2,       /* inconsistent shapes (Hq % Hkv != 0, cap < K, ...)      */
+  ORTHRUS_EUNSUPPORTED = -3, /* valid but not implemented (head_dim not 64/128, ...)  */
+  ORTHRUS_ECUDA = -4,        /* a CUDA runtime/driver call failed                     */
+  ORTHRUS_ECAPACITY = -5,    /* device: ctx_len + K would pass the cache capacity     */
+  ORTHRUS_EWORKSPACE = -6,   /* workspace missing or smaller than the size query says */
+  ORTHRUS_EALIGN = -7,       /* a pointer is not 16-byte aligned                      */
+  ORTHRUS_ETIMEOUT = -8      /* device: a bounded wait inside a kernel gave up        */
+} orthrus_status;
+
+typedef enum {
+  /* [GIST 2.2, 2.3 item 1] diffusion view: block row i sees keys [0, L+K):
+   * the whole committed prefix plus every block position, bidirectionally. */
+  ORTHRUS_MASK_DIFF = 0,
+  /* [GIST 2.3 item 2; HN #21] AR view: block row i sees keys [0, L+i+1):
+   * the prefix plus block positions 0..i.  K = 1 is ordinary decoding. */
+  ORTHRUS_MASK_AR = 1
+} orthrus_mask_mode;
+
+/*
+ * One layer's view of the shared KV cache ([GIST 2.1, 3]; [ABS]).
+ *   k, v      bf16 [B, Hkv, cap, d] device.  Slots [0, ctx_lens[b]) hold the
+ *             committed prefix of sequence b; before block attention the
+ *             caller writes the block's K/V (either view's projections) into
+ *             slots [ctx_lens[b], ctx_lens[b] + K).  Slots beyond that are
+ *             never read and may hold anything, including NaN.
+ *   ctx_lens  int32 [B] device: committed length L_b per sequence.  One array
+ *             serves all layers; orthrus_kv_commit advances it once per step.
+ * Rows of k and v (d * 2 bytes) and the base pointers must be 16-byte aligned.
+ */
+typedef struct {
+  void *k;
+  void *v;
+  int32_t *ctx_lens;
+  int B;
+  int Hkv;
+  int cap;
+  int d;
+} orthrus_kv_cache;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *orthrus_status_str(int status);
+
+/* ABI version of this header/library pair (incremented on any change). */
+int orthrus_abi_version(void);
+
+/*
+ * Workspace bytes orthrus_block_attn needs on the CURRENT device for these
+ * shapes (split-KV partial results; independent of the context lengths).
+ * Returns ORTHRUS_OK and writes *bytes, or a validation error.
+ */
+int orthrus_block_attn_workspace_size(int B, int Hq, int Hkv, int d, int K, size_t *bytes);
+
+/*
+ * Block-query attention over the shared KV cache ([GIST 2.1-2.3 items 1-2]).
+ *
+ * For sequence b, block row i in [0, K), query head h in [0, Hq), KV head
+ * g = h / (Hq / Hkv) (contiguous GQA groups):
+ *     s_j = (q[b,i,h,:] . k[b,g,j,:]) / sqrt(d)  for j < e,
+ *     e   = L_b + K        (ORTHRUS_MASK_DIFF)
+ *     e   = L_b + i + 1    (ORTHRUS_MASK_AR)
+ *     out[b,i,h,:] = sum_j softmax(s)_j * v[b,g,j,:]
+ * with bf16 inputs, fp32 accumulation and softmax, bf16 output.
+ *
+ *   q          bf16 [B, K, Hq, d] device (post-RoPE queries)
+ *   cache      KV cache view (host struct; its pointers are device pointers)
+ *   Hq, K      query heads (multiple of cache->Hkv), block size 1..32
+ *   mask_mode  orthrus_mask_mode
+ *   out        bf16 [B, K, Hq, d] device
+ *   workspace  device, >= orthrus_block_attn_workspace_size(...) bytes, any
+ *              contents; calls that share a workspace must be stream-ordered
+ *   dev_status int32 device or NULL (see conventions; ORTHRUS_ECAPACITY when
+ *              L_b + K > cap, in which case L_b is clamped to cap - K)
+ * Supported: d in {64, 128}; 1 <= K <= 32; Hq / Hkv <= 128.
+ * Runs as a persistent split-KV kernel (one CTA per SM, tcgen05 MMAs with TMEM
+ * accumulators, TMA-staged K/V tiles) followed by a log-sum-exp combine.
+ */
+int orthrus_block_attn(const void *q, const orthrus_kv_cache *cache, int Hq, int K,
+                       int mask_mode, void *out, void *workspace, size_t ws_bytes,
+                       int32_t *dev_status, void *stream);
+
+/*
+ * Workspace bytes orthrus_lmhead_argmax needs on the CURRENT device.
+ */
+int orthrus_lmhead_workspace_size(int R, int V, size_t *bytes);
+
+/*
+ * LM head with fused greedy choice ([GIST 2.3 items 2-3]: the frozen AR head
+ * gives the target at all K positions; a draft is kept only if it equals the
+ * greedy prediction).
+ *     logits[r, v] = sum_k h[r,k] * W[v,k]   (fp32 accumulation of bf16 products)
+ *     argmax[r]    = smallest v attaining max_v logits[r, v]
+ * The logits never reach HBM: the argmax is reduced in the GEMM epilogue.
+ *
+ *   h          bf16 [R, H] device (final hidden states of the R = B*K rows)
+ *   W          bf16 [V, H] device (nn.Linear weight layout)
+ *   argmax     int32 [R] device (output)
+ *   max_logit  fp32 [R] device or NULL (output: the maximum logit per row)
+ *   workspace  device, >= orthrus_lmhead_workspace_size(R, V) bytes
+ * Supported: 1 <= R; H % 64 == 0; 1 <= V < 2^31.  Rows are processed in
+ * passes of at most 256.
+ */
+int orthrus_lmhead_argmax(const void *h, const void *W, int R, int H, int V, int32_t *argmax,
+                          float *max_logit, void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Greedy choice over precomputed fp32 logits (a test helper for verifying
+ * from given logits).  logits fp32 [R, V] device -> argmax int32 [R] device
+ * (smallest index of the maximum; NaN entries are never chosen).
+ */
+int orthrus_row_argmax_f32(const float *logits, int R, int V, int32_t *argmax, void *stream);
+
+/*
+ * Exact consensus ([GIST 2.3 item 3]; [HN #21]).
+ * argmax[b,i] is the AR greedy token predicted by block row i (the token after
+ * block position i); draft[b,i] is the drafted token for the same position.
+ *     accept_len[b] = min { i : draft[b,i] != argmax[b,i] }, or K if none
+ *     next_tok[b]   = argmax[b, accept_len[b]]  if accept_len[b] < K
+ *                     draft[b, K-1]             otherwise
+ * next_tok is the new anchor (last emitted token, not yet in the cache).
+ *   argmax, draft  int32 [B, K] device;  accept_len, next_tok int32 [B] device.
+ * Supported: 1 <= K <= 32.  One warp per sequence, bit-exact.
+ */
+int orthrus_verify(const int32_t *argmax, const int32_t *draft, int B, int K,
+                   int32_t *accept_len, int32_t *next_tok, void *stream);
+
+/*
+ * KV commit by moving the length pointer ([GIST 2.3 item 3]: commit the
+ * synchronised prefix, shorten the cache; [ABS]: O(1) overhead).
+ * The verify pass cached the anchor and draft[0..K-2] in slots [L, L+K); the
+ * anchor plus the accepted drafts stay, so
+ *     ctx_lens[b] += min(accept_len[b] + 1, K)
+ * No KV element is moved or cleared: rejected slots are overwritten by the
+ * next block.  A length that would pass cache->cap is clamped to cap
+ * (ORTHRUS_ECAPACITY in dev_status); an accept length outside [0, K] leaves
+ * the length unchanged (ORTHRUS_EINVAL in dev_status).
+ *   cache       host struct; uses cache->ctx_lens, cache->B, cache->cap
+ *   accept_len  int32 [B] device
+ */
+int orthrus_kv_commit(const orthrus_kv_cache *cache, const int32_t *accept_len, int K,
+                      int32_t *dev_status, void *stream);
+
+/*
+ * orthrus_verify followed by orthrus_kv_commit in one launch (one warp per
+ * sequence).  Same arguments and results as the two calls in sequence.
+ */
+int orthrus_verify_commit(const int32_t *argmax, const int32_t *draft, int B, int K,
+                          int32_t *accept_len, int32_t *next_tok,
+                          const orthrus_kv_cache *cache, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORTHRUS_H_ */

@@ -1,0 +1,72 @@
+// C-ABI plumbing: status strings, ABI version, tensor-map encoding and device
+// queries shared by the kernels' host launchers.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "host.h"
+
+namespace orthrus {
+
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void resolve_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess) {
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+}
+}  // namespace
+
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box) {
+  std::call_once(g_encode_once, resolve_encode);
+  if (g_encode == nullptr) return ORTHRUS_ECUDA;
+  cuuint64_t gdim[5];
+  cuuint64_t gstride[4];
+  cuuint32_t bdim[5];
+  cuuint32_t estride[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+    if (i + 1 < rank) gstride[i] = strides_bytes[i];
+  }
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+                        const_cast<void*>(base), gdim, gstride, bdim, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ORTHRUS_OK : ORTHRUS_EINVAL;
+}
+
+int current_sm_count(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return ORTHRUS_ECUDA;
+  return ORTHRUS_OK;
+}
+
+}  // namespace orthrus
+
+extern "C" const char* orthrus_status_str(int status) {
+  switch (status) {
+    case ORTHRUS_OK: return "ORTHRUS_OK";
+    case ORTHRUS_EINVAL: return "ORTHRUS_EINVAL: invalid argument";
+    case ORTHRUS_ESHAPE: return "ORTHRUS_ESHAPE: inconsistent shapes";
+    case ORTHRUS_EUNSUPPORTED: return "ORTHRUS_EUNSUPPORTED: unsupported configuration";
+    case ORTHRUS_ECUDA: return "ORTHRUS_ECUDA: CUDA call failed";
+    case ORTHRUS_ECAPACITY: return "ORTHRUS_ECAPACITY: KV cache capacity exceeded";
+    case ORTHRUS_EWORKSPACE: return "ORTHRUS_EWORKSPACE: workspace missing or too small";
+    case ORTHRUS_EALIGN: return "ORTHRUS_EALIGN: pointer not 16-byte aligned";
+    case ORTHRUS_ETIMEOUT: return "ORTHRUS_ETIMEOUT: bounded device wait gave up";
+    default: return "ORTHRUS: unknown status";
+  }
+}
+
+extern "C" int orthrus_abi_version(void) { return 1; }

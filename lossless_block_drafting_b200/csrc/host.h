@@ -1,0 +1,28 @@
+// Host-side helpers shared by the C-ABI entry points: TMA tensor-map
+// encoding (through the driver entry point, so no -lcuda link is needed),
+// device queries and argument checks.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "orthrus.h"
+
+namespace orthrus {
+
+// Encode a bf16 tiled tensor map with 128-byte swizzle.  dims/strides follow
+// the driver API (dims[0] innermost; strides in bytes for dims 1..rank-1).
+// Returns ORTHRUS_OK, ORTHRUS_ECUDA (entry point missing) or ORTHRUS_EINVAL.
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box);
+
+// Number of SMs of the current device (ORTHRUS_ECUDA on failure).
+int current_sm_count(int* sms);
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace orthrus
