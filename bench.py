@@ -1,0 +1,575 @@
+"""Benchmark of the Orthrus dual-view decode step's hot path on B200.
+
+One step = one full decode step of the hot path on Qwen3-8B-shaped synthetic
+data (36 layers, 32 query / 8 KV heads, head_dim 128, hidden 4096, vocab
+151936), batch 1, block K = 32, context 40960:
+    diffusion pass: 36 x block attention (diffusion mask) + LM head argmax -> drafts
+    AR pass:        36 x block attention (AR mask)        + LM head argmax
+    consensus:      verify + KV commit (one launch)
+Metric: verified draft tokens per second = B*K / step time.  The step is
+captured once into a CUDA graph of K unrolled steps with event nodes at the
+phase boundaries, so the attention launches' average duration is measured on
+the launching stream inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+                    [--ctx L] [--block K] [--layers N] [--sweep]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (the reference arm of this benchmark).  Under torchrun (N > 1) every
+rank runs an independent replica (weak scaling: the path has no exchange
+step); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "verified draft tokens/sec per step at 40K ctx; attn HBM GB/s vs peak"
+UNIT = "tokens/s"
+QWEN = dict(Hq=32, Hkv=8, d=128, H=4096, V=151936, layers=36)
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ctx", type=int, default=40960)
+    ap.add_argument("--block", type=int, default=32)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--layers", type=int, default=QWEN["layers"])
+    ap.add_argument("--accept", type=int, default=4,
+                    help="planted accepted length per step (drafts agree with the AR "
+                         "argmax on this many leading rows)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also time K in {1,4,8,16,32} x L in {1024,8192,40960,131072}")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(
+            p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- workload
+class Workload:
+    """Resident synthetic inputs for one replica of the decode step."""
+
+    def __init__(self, B, K, L, layers, accept, steps_total, device, seed=0):
+        import torch
+        from lossless_block_drafting_b200 import orthrus as ob
+        self.ob = ob
+        self.B, self.K, self.L0, self.layers = B, K, L, layers
+        Hq, Hkv, d, H, V = QWEN["Hq"], QWEN["Hkv"], QWEN["d"], QWEN["H"], QWEN["V"]
+        self.Hq, self.Hkv, self.d, self.H, self.V = Hq, Hkv, d, H, V
+        # room for the committed length to grow by up to K per step
+        self.cap = L + K * (steps_total + 2)
+        g = torch.Generator(device=device).manual_seed(seed)
+        bf = torch.bfloat16
+
+        def randn(*shape, std=1.0):
+            x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+            return (x * std).to(bf) if std != 1.0 else x.to(bf)
+
+        self.k = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
+        self.v = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
+        self.q_diff = [randn(B, K, Hq, d) for _ in range(layers)]
+        self.q_ar = [randn(B, K, Hq, d) for _ in range(layers)]
+        self.W = randn(V, H, std=0.02)
+        self.h_ar = randn(B * K, H)
+        # the diffusion view's final states agree with the AR view's on the first
+        # `accept` rows of every block, so drafts match the AR argmax there
+        self.h_diff = randn(B * K, H)
+        a = max(0, min(accept, K))
+        hv = self.h_diff.view(B, K, H)
+        hv[:, :a] = self.h_ar.view(B, K, H)[:, :a]
+        self.accept = a
+        self.ctx_lens = torch.full((B,), L, dtype=torch.int32, device=device)
+        self.ctx_init = self.ctx_lens.clone()
+        self.attn_out = torch.empty(B, K, Hq, d, dtype=bf, device=device)
+        self.ws_attn = torch.empty(ob.block_attn_workspace_size(B, Hq, Hkv, d, K),
+                                   dtype=torch.uint8, device=device)
+        self.ws_lm = torch.empty(ob.lmhead_workspace_size(B * K, V), dtype=torch.uint8,
+                                 device=device)
+        self.draft = torch.empty(B * K, dtype=torch.int32, device=device)
+        self.argmax = torch.empty(B * K, dtype=torch.int32, device=device)
+        self.accept_len = torch.empty(B, dtype=torch.int32, device=device)
+        self.next_tok = torch.empty(B, dtype=torch.int32, device=device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.views = [ob.kv_cache_view(self.k[i], self.v[i], self.ctx_lens) for i in range(layers)]
+
+    # kernels launched per step (main + combine per attention call; main +
+    # reduce per LM head; one verify+commit)
+    @property
+    def launches_per_step(self):
+        return 2 * self.layers * 2 + 2 * 2 + 1
+
+    def attn_bytes(self):
+        """Algorithmic bytes of one attention call at the starting context."""
+        kv = 2 * self.B * self.Hkv * self.d * 2 * (self.L0 + self.K)
+        qo = 2 * self.B * self.K * self.Hq * self.d * 2
+        return kv + qo
+
+    def lm_bytes(self):
+        return self.V * self.H * 2 + self.B * self.K * self.H * 2
+
+    def step(self, stream, events=None):
+        """Issue one decode step on `stream`; events (if given) mark phase boundaries."""
+        ob = self.ob
+        ev = events or {}
+        if "t0" in ev:
+            ev["t0"].record(stream)
+        for i in range(self.layers):
+            ob.block_attn(self.q_diff[i], None, None, None, ob.MASK_DIFF, out=self.attn_out,
+                          workspace=self.ws_attn, dev_status=self.status, stream=stream,
+                          cache_view=self.views[i])
+        if "t1" in ev:
+            ev["t1"].record(stream)
+        ob.lmhead_argmax(self.h_diff, self.W, argmax=self.draft, workspace=self.ws_lm,
+                         stream=stream, dev_status=self.status)
+        if "t2" in ev:
+            ev["t2"].record(stream)
+        for i in range(self.layers):
+            ob.block_attn(self.q_ar[i], None, None, None, ob.MASK_AR, out=self.attn_out,
+                          workspace=self.ws_attn, dev_status=self.status, stream=stream,
+                          cache_view=self.views[i])
+        if "t3" in ev:
+            ev["t3"].record(stream)
+        ob.lmhead_argmax(self.h_ar, self.W, argmax=self.argmax, workspace=self.ws_lm,
+                         stream=stream, dev_status=self.status)
+        if "t4" in ev:
+            ev["t4"].record(stream)
+        ob.verify_commit(self.argmax.view(self.B, self.K), self.draft.view(self.B, self.K),
+                         self.ctx_lens, self.cap, accept_len=self.accept_len,
+                         next_tok=self.next_tok, dev_status=self.status, stream=stream)
+        if "t5" in ev:
+            ev["t5"].record(stream)
+
+
+def capture(wl: Workload, n_steps: int, stream, with_events: bool):
+    """CUDA graph of n_steps unrolled steps (+ external timing events per phase)."""
+    import torch
+    evs = []
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(n_steps):
+            e = None
+            if with_events:
+                e = {k: torch.cuda.Event(enable_timing=True, external=True)
+                     for k in ("t0", "t1", "t2", "t3", "t4", "t5")}
+                evs.append(e)
+            wl.step(stream, e)
+    return g, evs
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from lossless_block_drafting_b200 import build as libbuild
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    libbuild.build()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    hbm_peak, tc_peak, tc_sus, peak_kind = peaks()
+    K_steps, W_steps = args.steps, args.warmup
+    wl = Workload(args.batch, args.block, args.ctx, args.layers, args.accept,
+                  K_steps + W_steps + 4, dev, seed=1234 + rank)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        # eager warm-up (also loads the library and sets kernel attributes)
+        for _ in range(2):
+            wl.step(stream)
+        stream.synchronize()
+        g_warm, _ = capture(wl, 1, stream, with_events=False)
+        g_timed, evs = capture(wl, K_steps, stream, with_events=True)
+    wl.ctx_lens.copy_(wl.ctx_init)
+    torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(W_steps):
+            g_warm.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(dev.index)
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        g_timed.replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    ms_total = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / K_steps
+
+    # per-phase times from the event nodes of every timed step
+    ph = {"diff_attn": 0.0, "diff_lm": 0.0, "ar_attn": 0.0, "ar_lm": 0.0, "verify": 0.0}
+    for e in evs:
+        ph["diff_attn"] += e["t0"].elapsed_time(e["t1"])
+        ph["diff_lm"] += e["t1"].elapsed_time(e["t2"])
+        ph["ar_attn"] += e["t2"].elapsed_time(e["t3"])
+        ph["ar_lm"] += e["t3"].elapsed_time(e["t4"])
+        ph["verify"] += e["t4"].elapsed_time(e["t5"])
+    ph = {k: v / K_steps for k, v in ph.items()}
+    attn_us = (ph["diff_attn"] + ph["ar_attn"]) * 1e3 / (2 * wl.layers)
+    lm_us = (ph["diff_lm"] + ph["ar_lm"]) * 1e3 / 2
+    status = int(wl.status.item())
+
+    tokens = wl.B * wl.K
+    value = world * tokens / (ms_step * 1e-3)
+    attn_gbs = wl.attn_bytes() / (attn_us * 1e-6) / 1e9
+    lm_gbs = wl.lm_bytes() / (lm_us * 1e-6) / 1e9
+    lm_tflops = 2.0 * wl.B * wl.K * wl.H * wl.V / (lm_us * 1e-6) / 1e12
+    verify_pass_ms = ph["ar_attn"] + ph["ar_lm"] + ph["verify"]
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(wl, g_warm, stream, K_steps, W_steps, world, dev)
+
+    del g_timed, g_warm
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_steps,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/KV/hidden, N(0,0.02) LM head; "
+                "Qwen3-8B shapes, random weights)",
+        "config": {
+            "workload": f"qwen3-8b-shaped dual-view decode step: {wl.layers} layers, "
+                        f"batch {wl.B}, K {wl.K}, context {wl.L0}",
+            "step": "diffusion pass (36x block_attn DIFF + lmhead_argmax) + AR pass "
+                    "(36x block_attn AR + lmhead_argmax) + verify_commit",
+            "batch": wl.B, "block_K": wl.K, "ctx": wl.L0, "layers": wl.layers,
+            "heads": "32q/8kv d128", "hidden": wl.H, "vocab": wl.V,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (per step: "
+                  f"{(2 * wl.layers * wl.attn_bytes() + 2 * wl.lm_bytes()) / 1e9:.1f} GB read)",
+            "graph": "K steps unrolled in one CUDA graph",
+            "planted_accept_len": wl.accept,
+        },
+        "breakdown_ms_per_step": {k: round(v, 4) for k, v in ph.items()},
+        "verify_pass_only": {
+            "ms": round(verify_pass_ms, 4),
+            "tokens_per_s": round(world * tokens / (verify_pass_ms * 1e-3), 2),
+        },
+        "attn": {"us_per_call": round(attn_us, 2), "GB_per_s": round(attn_gbs, 1),
+                 "frac_of_hbm_peak": round(attn_gbs / hbm_peak, 4)},
+        "lmhead": {"us_per_call": round(lm_us, 2), "GB_per_s": round(lm_gbs, 1),
+                   "TFLOP_per_s": round(lm_tflops, 1),
+                   "frac_of_hbm_peak": round(lm_gbs / hbm_peak, 4),
+                   "frac_of_bf16_peak": round(lm_tflops / tc_sus, 4)},
+        "roofline": {
+            "kernel": "orthrus_block_attn (split-KV main + LSE combine), AR and DIFF masks",
+            "bound": "hbm",
+            "achieved": round(attn_gbs, 1),
+            "peak": hbm_peak,
+            "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
+                           if peak_kind == "measured" else "fallback 6650 GB/s",
+            "unit": "GB/s",
+            "frac": round(attn_gbs / hbm_peak, 4),
+            "traffic": None,
+            "algorithmic_bytes_per_launch": wl.attn_bytes(),
+        },
+        "gpu_launches": wl.launches_per_step * K_steps,
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl.L0, wl.K, wl.layers)
+    if args.sweep and rank == 0:
+        result["sweep"] = run_sweep(dev, stream)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):
+    """Same metric end to end: per step, H2D of the step's inputs from pinned host
+    memory, the captured step (public C-ABI calls), and a D2H read of the results."""
+    import torch
+    host_in = []
+    for i in range(wl.layers):
+        host_in.append((wl.q_diff[i].cpu().pin_memory(), wl.q_diff[i]))
+        host_in.append((wl.q_ar[i].cpu().pin_memory(), wl.q_ar[i]))
+    host_in.append((wl.h_diff.cpu().pin_memory(), wl.h_diff))
+    host_in.append((wl.h_ar.cpu().pin_memory(), wl.h_ar))
+    outs = [wl.accept_len, wl.next_tok, wl.ctx_lens]
+    host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    def one():
+        with torch.cuda.stream(stream):
+            for h, d in host_in:
+                d.copy_(h, non_blocking=True)
+            g_step.replay()
+            for h, d in zip(host_out, outs):
+                h.copy_(d, non_blocking=True)
+        stream.synchronize()
+
+    wl.ctx_lens.copy_(wl.ctx_init)
+    for _ in range(W_steps):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    t0 = time.perf_counter()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(K_steps):
+        one()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / K_steps
+    wall_ms = (time.perf_counter() - t0) * 1e3 / K_steps
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": round(world * wl.B * wl.K / (ms * 1e-3), 2), "unit": UNIT,
+            "ms_per_step": round(ms, 4), "host_wall_ms_per_step": round(wall_ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+def run_sweep(dev, stream):
+    """Config 5 sweep: AR-pass step time for K x L (36 layers, batch 1)."""
+    import torch
+    out = []
+    for L in (1024, 8192, 40960, 131072):
+        for K in (1, 4, 8, 16, 32):
+            layers = QWEN["layers"]
+            wl = Workload(1, K, L, layers, 0, 12, dev, seed=7)
+            with torch.cuda.stream(stream):
+                wl.step(stream)
+                stream.synchronize()
+                g, evs = capture(wl, 5, stream, with_events=True)
+            with torch.cuda.stream(stream):
+                for _ in range(2):
+                    wl.ctx_lens.copy_(wl.ctx_init)
+                    g.replay()
+            torch.cuda.synchronize()
+            ar = sum(e["t2"].elapsed_time(e["t3"]) for e in evs) / len(evs)
+            lm = sum(e["t3"].elapsed_time(e["t4"]) for e in evs) / len(evs)
+            vc = sum(e["t4"].elapsed_time(e["t5"]) for e in evs) / len(evs)
+            full = sum(e["t0"].elapsed_time(e["t5"]) for e in evs) / len(evs)
+            attn_us = ar * 1e3 / layers
+            out.append({"ctx": L, "K": K,
+                        "verify_step_ms": round(ar + lm + vc, 4),
+                        "full_step_ms": round(full, 4),
+                        "attn_us": round(attn_us, 2),
+                        "attn_GB_per_s": round(wl.attn_bytes() / (attn_us * 1e-6) / 1e9, 1),
+                        "verified_tok_per_s": round(K / ((ar + lm + vc) * 1e-3), 1)})
+            del g, evs, wl
+            torch.cuda.empty_cache()
+    return out
+
+
+# -------------------------------------------------------------- CPU oracle
+class OracleSample:
+    """The fp64 oracle timed on a bounded sample of one step, scaled to a step.
+
+    Sample: AR-mask attention of ONE KV head (its 4 query heads x K rows) of one
+    layer at context L, and the LM head for `lm_rows` of the K hidden rows.
+    Scaled: attention x (8 KV heads x layers x 2 passes), LM head x (K/lm_rows x 2).
+    """
+
+    def __init__(self, L, K, layers, lm_rows=8, seed=0):
+        from lossless_block_drafting_b200 import synth
+        self.L, self.K, self.layers, self.lm_rows = L, K, layers, lm_rows
+        self.case = synth.attn_case(1, K, 4, 1, 128, [L], seed=seed, poison=None)
+        self.h, self.W = synth.lmhead_case(lm_rows, QWEN["H"], QWEN["V"], seed=seed)
+
+    def run(self):
+        import numpy as np
+
+        import oracle
+        c = self.case
+        t0 = time.perf_counter()
+        oracle.block_attn(c.q, c.k_cache, c.v_cache, c.ctx_lens, oracle.MASK_AR)
+        t_attn = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        am, _, _ = oracle.lmhead_argmax(self.h, self.W)
+        t_lm = time.perf_counter() - t0
+        blk = np.asarray([np.resize(am, self.K)])
+        t0 = time.perf_counter()
+        oracle.verify(blk, blk)
+        t_v = time.perf_counter() - t0
+        t_step = (t_attn * QWEN["Hkv"] * self.layers * 2 + t_lm * (self.K / self.lm_rows) * 2
+                  + t_v)
+        return {"t_attn_sample_s": t_attn, "t_lm_sample_s": t_lm, "t_step_s": t_step,
+                "threads": oracle.num_threads()}
+
+    def describe(self, r):
+        return (f"fp64 C oracle: AR attention of 1 of 8 KV heads of 1 layer at ctx {self.L} "
+                f"({r['t_attn_sample_s']:.2f} s) + LM head for {self.lm_rows} of {self.K} rows "
+                f"({r['t_lm_sample_s']:.2f} s), scaled to 2 passes x {self.layers} layers x 8 "
+                f"KV heads and 2 x {self.K} LM-head rows (step {r['t_step_s']:.1f} s)")
+
+
+def cpu_baseline(L, K, layers):
+    s = OracleSample(L, K, layers)
+    r = s.run()
+    return {"value": round(K / r["t_step_s"], 4), "unit": UNIT, "cores": r["threads"],
+            "kind": "oracle", "sample": s.describe(r)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    L, K, layers = args.ctx, args.block, args.layers
+    s = OracleSample(L, K, layers)
+    for _ in range(args.warmup):
+        s.run()
+    rs = [s.run() for _ in range(args.steps)]
+    t_step = statistics.mean(r["t_step_s"] for r in rs)
+    value = args.batch * K / t_step
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(t_step * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"qwen3-8b-shaped dual-view decode step: {layers} layers, "
+                               f"batch {args.batch}, K {K}, context {L}",
+                   "reference": "fp64 CPU oracle (the pages publish no code to run)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "kind": "oracle",
+                         "cores": oracle.num_threads(), "sample": s.describe(rs[-1])},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if res is not None:
+        line = json.dumps(res)
+        print(line, flush=True)
+        if args.json_out:
+            with open(args.json_out, "w") as f:
+                f.write(line + "\n")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -145,11 +145,13 @@ int orthrus_lmhead_workspace_size(int R, int V, size_t *bytes);
  *   argmax     int32 [R] device (output)
  *   max_logit  fp32 [R] device or NULL (output: the maximum logit per row)
  *   workspace  device, >= orthrus_lmhead_workspace_size(R, V) bytes
+ *   dev_status int32 device or NULL (ORTHRUS_ETIMEOUT if a bounded wait gave up)
  * Supported: 1 <= R; H % 64 == 0; 1 <= V < 2^31.  Rows are processed in
  * passes of at most 256.
  */
 int orthrus_lmhead_argmax(const void *h, const void *W, int R, int H, int V, int32_t *argmax,
-                          float *max_logit, void *workspace, size_t ws_bytes, void *stream);
+                          float *max_logit, void *workspace, size_t ws_bytes,
+                          int32_t *dev_status, void *stream);
 
 /*
  * Greedy choice over precomputed fp32 logits (a test helper for verifying

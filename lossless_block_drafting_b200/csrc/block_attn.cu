@@ -13,18 +13,20 @@
 // all (sequence, KV head) segments is cut into 64-key tiles and spread evenly
 // over a persistent grid of one CTA per SM (split-KV / flash-decoding); a
 // CTA's contiguous tile range may cross segment boundaries and then emits one
-// partial result per segment piece.  Per CTA:
-//   warp 0      TMA producer: Q tile per piece, K and V tiles into a 4-stage
-//               ring (128-byte swizzle).
-//   warp 1      tcgen05 issuer: S = Q K^T into one of two TMEM buffers, then
-//               O += P V into a TMEM accumulator (V read MN-major).
-//   warp 2      TMEM allocation.
-//   warps 4-7   softmax, one thread per row: S from TMEM, mask, online
-//               softmax in the exp2 domain (rescaling O in TMEM only when the
-//               running max grows by more than 2^8, which is exact because
-//               the final normaliser uses the same reference), P as bf16 into
-//               swizzled shared memory, and the piece epilogue writing
-//               (O, m, l) partials.
+// partial result per segment piece.  Per CTA (12 warps), each single-thread
+// role on its own ring so no wait of one stream stalls another:
+//   warp 0      TMA: Q tile per piece, K tiles into a 4-stage ring.
+//   warp 2      TMA: V tiles into a 6-stage ring (V is held longer than K);
+//               the whole warp also allocates and frees TMEM.
+//   warp 1      tcgen05 issuer for S = Q K^T into TMEM buffer S_w.
+//   warp 3      tcgen05 issuer for O_w += P V (V read MN-major).
+//   warps 4-11  two softmax warpgroups taking alternate tiles, one thread per
+//               row: S from TMEM, mask, online softmax in the exp2 domain
+//               (rescaling O in TMEM only when the running max grows by more
+//               than 2^8, exact because the final normaliser uses the same
+//               reference), P as bf16 into swizzled shared memory.  At the end
+//               of a piece group 0 merges both groups' (m, l, O) and writes the
+//               piece's partial result.
 // A second, small kernel merges the partials of each segment by log-sum-exp
 // and writes bf16 output.
 #include <cuda_bf16.h>
@@ -38,11 +40,12 @@ namespace orthrus {
 namespace attn {
 
 constexpr int TN = 64;        // keys per tile
-constexpr int NS = 4;         // K and V ring stages
+constexpr int NK = 4;         // K ring stages (a K tile is released once S = Q K^T is done)
+constexpr int NV = 6;         // V ring stages (a V tile is held until O += P V is done)
 constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
-constexpr int THREADS = 256;
-constexpr int TMEM_COLS = 256;
-constexpr int TMEM_O = 128;   // column of the O accumulator (S buffers at 0 and TN)
+constexpr int THREADS = 384;  // 12 warps: TMA, MMA, TMEM alloc, spare, 2 softmax groups
+constexpr int TMEM_COLS = 512;
+constexpr int TMEM_O = 128;   // O accumulators at 128 and 256 (S buffers at 0 and TN)
 
 template <int D>
 struct Layout {
@@ -54,10 +57,11 @@ struct Layout {
   static constexpr int P_BYTES = ROWS * TN * 2;     // one 128-byte chunk per row
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int NBAR = 4 * NS + 13;
+  static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + NV * KV_BYTES;
+  static constexpr int OFF_ML = OFF_P + 2 * P_BYTES;   // [ROWS] float2 handed WG1 -> WG0
+  static constexpr int OFF_BAR = OFF_ML + ROWS * 8;
+  static constexpr int NBAR = 2 * NK + 2 * NV + 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
@@ -136,10 +140,13 @@ __device__ __forceinline__ long long cta_of(long long x, long long T, long long 
 
 // Wait that ignores the abort flag, used only to drain in-flight async work
 // before the CTA exits.
-__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int32_t* status) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) return;  // 200 ms
+    if (globaltimer_ns() - t0 > 200000000ull) {  // 200 ms
+      report(status, ORTHRUS_ETIMEOUT);
+      return;
+    }
   }
 }
 
@@ -160,20 +167,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const uint32_t bar = sb0 + Ly::OFF_BAR;
   auto full_k = [&](int s) { return bar + 8u * s; };
-  auto full_v = [&](int s) { return bar + 8u * (NS + s); };
-  auto empty_k = [&](int s) { return bar + 8u * (2 * NS + s); };
-  auto empty_v = [&](int s) { return bar + 8u * (3 * NS + s); };
-  const uint32_t q_full = bar + 8u * (4 * NS + 0);
-  const uint32_t q_empty = bar + 8u * (4 * NS + 1);
-  auto s_full = [&](int i) { return bar + 8u * (4 * NS + 2 + i); };
-  auto s_free = [&](int i) { return bar + 8u * (4 * NS + 4 + i); };
-  auto p_full = [&](int i) { return bar + 8u * (4 * NS + 6 + i); };
-  auto p_empty = [&](int i) { return bar + 8u * (4 * NS + 8 + i); };
-  const uint32_t o_full = bar + 8u * (4 * NS + 10);
-  const uint32_t o_free = bar + 8u * (4 * NS + 11);
-  const uint32_t mma_done = bar + 8u * (4 * NS + 12);
+  auto empty_k = [&](int s) { return bar + 8u * (NK + s); };
+  auto full_v = [&](int s) { return bar + 8u * (2 * NK + s); };
+  auto empty_v = [&](int s) { return bar + 8u * (2 * NK + NV + s); };
+  const uint32_t bar2 = bar + 8u * (2 * NK + 2 * NV);
+  const uint32_t q_full = bar2;
+  const uint32_t q_empty = bar2 + 8u;
+  auto s_full = [&](int i) { return bar2 + 8u * (2 + i); };
+  auto s_free = [&](int i) { return bar2 + 8u * (4 + i); };
+  auto p_full = [&](int i) { return bar2 + 8u * (6 + i); };
+  auto p_empty = [&](int i) { return bar2 + 8u * (8 + i); };
+  const uint32_t o_full = bar2 + 8u * 10;
+  const uint32_t o_free = bar2 + 8u * 11;
+  const uint32_t mma_done = bar2 + 8u * 12;  // both MMA issuers commit once at exit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
+  float2* ml_xchg = reinterpret_cast<float2*>(smem + Ly::OFF_ML);
 
   const long long T = total_tiles(p, blockIdx.x == 0 && threadIdx.x == 0);
   const long long Pc = gridDim.x;
@@ -182,10 +191,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n = static_cast<int>(x1 - x0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(full_k(s), 1);
-      mbar_init(full_v(s), 1);
       mbar_init(empty_k(s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(full_v(s), 1);
       mbar_init(empty_v(s), 1);
     }
     mbar_init(q_full, 1);
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, 4);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -218,14 +229,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (!mbar_wait_warp((barrier), (parity), abort_flag, p.dev_status)) on_fail
 
   if (n > 0 && warp == 0 && lane == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------- Q and K producer
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
     const uint64_t policy = policy_evict_first();
     Cursor cur;
     cursor_seek(cur, p, x0);
-    int pieces = 0, issued_k = 0, issued_v = 0;
+    int pieces = 0, issued = 0;
     const uint32_t q_tx = static_cast<uint32_t>(p.Gc * p.K * D * 2);
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cur.t == 0;
@@ -238,49 +248,61 @@ __global__ void __launch_bounds__(THREADS, 1)
                       g * p.G + hc * p.Gc, cur.b * p.K);
         ++pieces;
       }
-      const int stage = j % NS;
-      const uint32_t ph = (j / NS) & 1;
+      const int stage = j % NK;
       const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
-      WAIT_OR(empty_k(stage), ph ^ 1, break);
+      WAIT_OR(empty_k(stage), ((j / NK) & 1) ^ 1, break);
       mbar_arrive_expect_tx(full_k(stage), Ly::KV_BYTES);
       for (int c = 0; c < Ly::CHUNKS; ++c)
         tma_load_2d_hint(sb0 + Ly::OFF_K + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK, &tmK,
                          full_k(stage), c * 64, row0, policy);
-      ++issued_k;
-      WAIT_OR(empty_v(stage), ph ^ 1, break);
+      ++issued;
+      cursor_next(cur, p);
+    }
+    // Drain: every issued copy must have landed before the CTA may exit.
+    for (int j = (issued > NK ? issued - NK : 0); j < issued; ++j)
+      mbar_wait_drain(full_k(j % NK), (j / NK) & 1, p.dev_status);
+    if (pieces > 0) mbar_wait_drain(q_full, (pieces - 1) & 1, p.dev_status);
+  } else if (n > 0 && warp == 2 && lane == 0) {
+    // ------------------------------------------------------- V producer
+    prefetch_tmap(&tmV);
+    const uint64_t policy = policy_evict_first();
+    Cursor cur;
+    cursor_seek(cur, p, x0);
+    int issued = 0;
+    for (int j = 0; j < n; ++j) {
+      const int g = cur.seg / p.nhc;
+      const int stage = j % NV;
+      const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
+      WAIT_OR(empty_v(stage), ((j / NV) & 1) ^ 1, break);
       mbar_arrive_expect_tx(full_v(stage), Ly::KV_BYTES);
       for (int c = 0; c < Ly::CHUNKS; ++c)
         tma_load_2d_hint(sb0 + Ly::OFF_V + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK, &tmV,
                          full_v(stage), c * 64, row0, policy);
-      ++issued_v;
+      ++issued;
       cursor_next(cur, p);
     }
-    // Drain: every issued copy must have landed before the CTA may exit.
-    for (int j = (issued_k > NS ? issued_k - NS : 0); j < issued_k; ++j)
-      mbar_wait_drain(full_k(j % NS), (j / NS) & 1);
-    for (int j = (issued_v > NS ? issued_v - NS : 0); j < issued_v; ++j)
-      mbar_wait_drain(full_v(j % NS), (j / NS) & 1);
-    if (pieces > 0) mbar_wait_drain(q_full, (pieces - 1) & 1);
+    for (int j = (issued > NV ? issued - NV : 0); j < issued; ++j)
+      mbar_wait_drain(full_v(j % NV), (j / NV) & 1, p.dev_status);
   } else if (n > 0 && warp == 1 && lane == 0) {
-    // -------------------------------------------------------- MMA issuer
+    // ------------------------------------------------ S = Q K^T issuer
+    // Tile j belongs to softmax warpgroup w = j & 1 and lands in TMEM S_w.
     const uint32_t id_s = make_idesc_bf16_f32(ROWS, TN, false, false);
-    const uint32_t id_pv = make_idesc_bf16_f32(ROWS, D, false, true);
-    Cursor cs, cp;
+    Cursor cs;
     cursor_seek(cs, p, x0);
-    cursor_seek(cp, p, x0);
-    int q_seen = 0, pieces_done = 0;
-    auto issue_s = [&](int j) -> bool {
+    int q_seen = 0;
+    for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cs.t == 0;
       const bool last = (j == n - 1) || cs.t == cs.nt - 1;
       if (first) {
-        WAIT_OR(q_full, q_seen & 1, return false);
+        WAIT_OR(q_full, q_seen & 1, break);
         ++q_seen;
       }
-      const int stage = j % NS;
-      WAIT_OR(full_k(stage), (j / NS) & 1, return false);
-      const int sb = j & 1;
-      if (j >= 2) {
-        WAIT_OR(s_free(sb), ((j - 2) >> 1) & 1, return false);
+      const int stage = j % NK;
+      WAIT_OR(full_k(stage), (j / NK) & 1, break);
+      const int w = j & 1;
+      const int u = j >> 1;
+      if (u >= 1) {
+        WAIT_OR(s_free(w), (u - 1) & 1, break);
       }
       tc_fence_after();
       const uint32_t qa = sb0 + Ly::OFF_Q;
@@ -291,38 +313,49 @@ __global__ void __launch_bounds__(THREADS, 1)
                                        kSwizzle128B);
         const uint64_t bd = make_sdesc(ka + (kk >> 2) * Ly::KV_CHUNK + (kk & 3) * 32, 16, 1024,
                                        kSwizzle128B);
-        mma_bf16_ss(tmem + sb * TN, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + w * TN, ad, bd, id_s, kk > 0 ? 1u : 0u);
       }
       mma_commit(empty_k(stage));
-      mma_commit(s_full(sb));
+      mma_commit(s_full(w));
       if (last) mma_commit(q_empty);
       cursor_next(cs, p);
-      return true;
-    };
-    bool ok = issue_s(0);
-    for (int j = 0; ok && j < n; ++j) {
-      if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+    }
+    // every MMA of both issuers must be complete before TMEM is released
+    mma_commit(mma_done);
+    mbar_wait_drain(mma_done, 0, p.dev_status);
+  } else if (n > 0 && warp == 3 && lane == 0) {
+    // ------------------------------------------------ O_w += P V issuer
+    const uint32_t id_pv = make_idesc_bf16_f32(ROWS, D, false, true);
+    Cursor cp;
+    cursor_seek(cp, p, x0);
+    int pieces_done = 0, jp = 0;
+    for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cp.t == 0;
       const bool last = (j == n - 1) || cp.t == cp.nt - 1;
-      if (first && pieces_done > 0) {
-        WAIT_OR(o_free, (pieces_done - 1) & 1, break);
+      if (first) {
+        jp = j;
+        if (pieces_done > 0) {
+          WAIT_OR(o_free, (pieces_done - 1) & 1, break);
+        }
       }
-      WAIT_OR(p_full(j & 1), (j >> 1) & 1, break);
-      const int stage = j % NS;
-      WAIT_OR(full_v(stage), (j / NS) & 1, break);
+      const int w = j & 1;
+      WAIT_OR(p_full(w), (j >> 1) & 1, break);
+      const int stage = j % NV;
+      WAIT_OR(full_v(stage), (j / NV) & 1, break);
       tc_fence_after();
-      const uint32_t pa = sb0 + Ly::OFF_P + (j & 1) * Ly::P_BYTES;
+      const uint32_t pa = sb0 + Ly::OFF_P + w * Ly::P_BYTES;
       const uint32_t va = sb0 + Ly::OFF_V + stage * Ly::KV_BYTES;
+      const bool fresh = (j - jp) < 2;  // first tile of group w in this piece
 #pragma unroll
       for (int kk = 0; kk < TN / 16; ++kk) {
         const uint64_t ad = make_sdesc(pa + kk * 32, 16, 1024, kSwizzle128B);
         // V is [keys x d] with d contiguous: MN-major B operand.  16 keys per
         // step = two 8-row swizzle atoms (2048 B); d chunks Ly::KV_CHUNK apart.
         const uint64_t bd = make_sdesc(va + kk * 2048, Ly::KV_CHUNK, 1024, kSwizzle128B);
-        mma_bf16_ss(tmem + TMEM_O, ad, bd, id_pv, (first && kk == 0) ? 0u : 1u);
+        mma_bf16_ss(tmem + TMEM_O + w * 128, ad, bd, id_pv, (fresh && kk == 0) ? 0u : 1u);
       }
       mma_commit(empty_v(stage));
-      mma_commit(p_empty(j & 1));
+      mma_commit(p_empty(w));
       if (last) {
         mma_commit(o_full);
         ++pieces_done;
@@ -330,132 +363,161 @@ __global__ void __launch_bounds__(THREADS, 1)
       cursor_next(cp, p);
     }
     mma_commit(mma_done);
-    mbar_wait_drain(mma_done, 0);
+    mbar_wait_drain(mma_done, 0, p.dev_status);
   } else if (n > 0 && warp >= 4) {
     // ------------------------------------------------ softmax + epilogue
-    const int r = (warp - 4) * 32 + lane;
+    const int w = (warp - 4) >> 2;            // softmax warpgroup: even / odd tiles
+    const int r = (warp & 3) * 32 + lane;     // query row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t t_s = lane_base + w * TN;
+    const uint32_t t_o = lane_base + TMEM_O + w * 128;
     const int rows_valid = p.Gc * p.K;
     const int i_row = r / p.Gc;
+    const float sl2 = p.sl2;
     Cursor cur;
     cursor_seek(cur, p, x0);
-    int pieces = 0;
+    int pieces = 0, jp = 0;
     float m_used = -INFINITY, l_sum = 0.f;
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cur.t == 0;
       const bool last = (j == n - 1) || cur.t == cur.nt - 1;
       if (first) {
+        jp = j;
         m_used = -INFINITY;
         l_sum = 0.f;
       }
-      const int kv_end = cur.L + p.K;
-      const int lim = (r >= rows_valid) ? 0
-                      : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
-      const int tile0 = cur.t * TN;
-      const int sb = j & 1;
-      WARP_WAIT_OR(s_full(sb), (j >> 1) & 1, break);
-      tc_fence_after();
-      uint32_t ra[32], rb[32];
-      tmem_ld32(lane_base + sb * TN, ra);
-      tmem_ld32(lane_base + sb * TN + 32, rb);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free(sb));
-
-      float x[TN];
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < TN; ++c) {
-        const float s = __uint_as_float(c < 32 ? ra[c] : rb[c - 32]);
-        const float v = (tile0 + c < lim) ? s * p.sl2 : -INFINITY;
-        x[c] = v;
-        mx = fmaxf(mx, v);
-      }
-      float m_new = m_used;
-      if (first) {
-        m_new = mx;
-      } else if (__any_sync(0xFFFFFFFFu, mx > m_used + 8.f)) {
-        m_new = fmaxf(m_used, mx);
-        const float f = (m_new == -INFINITY) ? 1.f
-                        : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
-        // O may only be touched once the previous P*V has completed.
-        WARP_WAIT_OR(p_empty((j - 1) & 1), ((j - 1) >> 1) & 1, break);
+      if ((j & 1) == w) {
+        const bool fresh = (j - jp) < 2;
+        const int u = j >> 1;
+        const int kv_end = cur.L + p.K;
+        const int lim = (r >= rows_valid) ? 0
+                        : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+        const int tile0 = cur.t * TN;
+        WARP_WAIT_OR(s_full(w), u & 1, break);
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + TMEM_O + c0, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-          tmem_st32(lane_base + TMEM_O + c0, o);
-        }
-        tmem_wait_st();
-        l_sum *= f;
-      }
-      m_used = m_new;
-      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < TN; ++c) {
-        x[c] = fast_exp2(x[c] - m_eff);
-        rs += x[c];
-      }
-      l_sum += rs;
-
-      if (tile0 + TN > kv_end) {
-        // The tile runs past the valid keys: zero those V rows so that stale
-        // or NaN cache contents cannot reach O through 0 * NaN.
-        const int stage = j % NS;
-        WARP_WAIT_OR(full_v(stage), (j / NS) & 1, break);
-        const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
-        const int per_chunk = (TN - nv) * 8;
-        uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES;
-        for (int q = r; q < per_chunk * Ly::CHUNKS; q += ROWS) {
-          const int ch = q / per_chunk, rem = q % per_chunk;
-          *reinterpret_cast<uint4*>(vt + ch * Ly::KV_CHUNK + (nv + rem / 8) * 128 +
-                                    (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-      if (j >= 2) {
-        WARP_WAIT_OR(p_empty(sb), ((j - 2) >> 1) & 1, break);
-      }
-      uint8_t* prow = smem + Ly::OFF_P + sb * Ly::P_BYTES + r * 128;
-#pragma unroll
-      for (int pc = 0; pc < 8; ++pc) {
-        uint4 v;
-        v.x = pack_bf16x2(x[8 * pc + 0], x[8 * pc + 1]);
-        v.y = pack_bf16x2(x[8 * pc + 2], x[8 * pc + 3]);
-        v.z = pack_bf16x2(x[8 * pc + 4], x[8 * pc + 5]);
-        v.w = pack_bf16x2(x[8 * pc + 6], x[8 * pc + 7]);
-        *reinterpret_cast<uint4*>(prow + ((pc ^ (r & 7)) * 16)) = v;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(p_full(sb));
-
-      if (last) {
-        WARP_WAIT_OR(o_full, pieces & 1, break);
-        tc_fence_after();
-        const long long slot = static_cast<long long>(cur.b) * nseg + cur.seg + blockIdx.x;
-        float* dst = p.part_o + (slot * ROWS + r) * D;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + TMEM_O + c0, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; k += 4)
-            *reinterpret_cast<float4*>(dst + c0 + k) =
-                make_float4(__uint_as_float(o[k]), __uint_as_float(o[k + 1]),
-                            __uint_as_float(o[k + 2]), __uint_as_float(o[k + 3]));
-        }
-        p.part_ml[slot * ROWS + r] = make_float2(m_used, l_sum);
+        uint32_t ra[32], rb[32];
+        tmem_ld32(t_s, ra);
+        tmem_ld32(t_s + 32, rb);
+        tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(o_free);
+        if (lane == 0) mbar_arrive(s_free(w));
+
+        float x[TN];
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < TN; ++c) {
+          const float s = __uint_as_float(c < 32 ? ra[c] : rb[c - 32]);
+          const float v = (tile0 + c < lim) ? s : -INFINITY;
+          x[c] = v;
+          mx4[c & 3] = fmaxf(mx4[c & 3], v);
+        }
+        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        bool waited = false;
+        float m_new = m_used;
+        if (fresh) {
+          m_new = mx;
+        } else if (__any_sync(0xFFFFFFFFu, mx > m_used + 8.f)) {
+          m_new = fmaxf(m_used, mx);
+          const float f = (m_new == -INFINITY) ? 1.f
+                          : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
+          // O_w may only be touched once this group's previous P*V completed.
+          WARP_WAIT_OR(p_empty(w), (u - 1) & 1, break);
+          waited = true;
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(t_o + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+            tmem_st32(t_o + c0, o);
+          }
+          tmem_wait_st();
+          l_sum *= f;
+        }
+        m_used = m_new;
+        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < TN; ++c) {
+          x[c] = fast_exp2(fmaf(x[c], sl2, -m_eff));
+          rs4[c & 3] += x[c];
+        }
+        l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+
+        if (tile0 + TN > kv_end) {
+          // The tile runs past the valid keys: zero those V rows so that stale
+          // or NaN cache contents cannot reach O through 0 * NaN.
+          const int stage = j % NV;
+          WARP_WAIT_OR(full_v(stage), (j / NV) & 1, break);
+          const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
+          const int per_chunk = (TN - nv) * 8;
+          uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES;
+          for (int q = r; q < per_chunk * Ly::CHUNKS; q += ROWS) {
+            const int ch = q / per_chunk, rem = q % per_chunk;
+            *reinterpret_cast<uint4*>(vt + ch * Ly::KV_CHUNK + (nv + rem / 8) * 128 +
+                                      (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        if (u >= 1 && !waited) {
+          WARP_WAIT_OR(p_empty(w), (u - 1) & 1, break);
+        }
+        uint8_t* prow = smem + Ly::OFF_P + w * Ly::P_BYTES + r * 128;
+#pragma unroll
+        for (int pc = 0; pc < 8; ++pc) {
+          uint4 v;
+          v.x = pack_bf16x2(x[8 * pc + 0], x[8 * pc + 1]);
+          v.y = pack_bf16x2(x[8 * pc + 2], x[8 * pc + 3]);
+          v.z = pack_bf16x2(x[8 * pc + 4], x[8 * pc + 5]);
+          v.w = pack_bf16x2(x[8 * pc + 6], x[8 * pc + 7]);
+          *reinterpret_cast<uint4*>(prow + ((pc ^ (r & 7)) * 16)) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(w));
+      }
+
+      if (last) {
+        // Piece epilogue: merge the two groups' (m, l, O) and publish it.
+        WARP_WAIT_OR(o_full, pieces & 1, break);
+        tc_fence_after();
+        if (w == 1) ml_xchg[r] = make_float2(m_used, l_sum);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (w == 0) {
+          const float2 o1 = ml_xchg[r];
+          const float M = fmaxf(m_used, o1.x);
+          const float a0 = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
+          const float a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
+          const long long slot = static_cast<long long>(cur.b) * nseg + cur.seg + blockIdx.x;
+          float* dst = p.part_o + (slot * ROWS + r) * D;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o0[32], o1r[32];
+            tmem_ld32(t_o + c0, o0);
+            tmem_ld32(t_o + 128 + c0, o1r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+              float4 v;
+              v.x = (a0 != 0.f ? a0 * __uint_as_float(o0[k]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k]) : 0.f);
+              v.y = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 1]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 1]) : 0.f);
+              v.z = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 2]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
+              v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
+              *reinterpret_cast<float4*>(dst + c0 + k) = v;
+            }
+          }
+          p.part_ml[slot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
         ++pieces;
       }
       cursor_next(cur, p);
@@ -474,13 +536,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // Merge the pieces of each (sequence, KV head, head chunk) segment by
 // log-sum-exp.  One warp per query row; lane owns D/32 consecutive columns.
+// The pieces' (m, l) pairs are read lane-parallel and their O rows are
+// fetched with independent loads so the merge is bandwidth-, not
+// latency-bound.
 template <int D>
-__global__ void __launch_bounds__(256) attn_combine_kernel(const Params p, int grid_ctas,
+__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p, int grid_ctas,
                                                            __nv_bfloat16* __restrict__ out) {
   constexpr int PER = D / 32;
   const int s = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * 8 + warp;
+  const int r = blockIdx.y * 4 + warp;
   const int nseg = p.Hkv * p.nhc;
   const int b = s / nseg, seg = s % nseg;
   const int g = seg / p.nhc, hc = seg % p.nhc;
@@ -501,28 +566,49 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const Params p, int g
   const long long c0 = cta_of(Ts, T, P), c1 = cta_of(Ts + nt_b - 1, T, P);
 
   float M = -INFINITY;
-  for (long long c = c0; c <= c1; ++c) {
-    if (cta_start(c, T, P) == cta_start(c + 1, T, P)) continue;
-    M = fmaxf(M, p.part_ml[(s + c) * ROWS + r].x);
+  for (long long base = c0; base <= c1; base += 32) {
+    const long long c = base + lane;
+    if (c <= c1 && cta_start(c, T, P) != cta_start(c + 1, T, P))
+      M = fmaxf(M, __ldcg(&p.part_ml[(s + c) * ROWS + r]).x);
   }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, m));
+
   float acc[PER];
 #pragma unroll
   for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  float L = 0.f;
-  for (long long c = c0; c <= c1; ++c) {
-    if (cta_start(c, T, P) == cta_start(c + 1, T, P)) continue;
-    const float2 ml = p.part_ml[(s + c) * ROWS + r];
-    const float w = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-    L += w * ml.y;
-    const float* src = p.part_o + ((s + c) * ROWS + r) * D + lane * PER;
-#pragma unroll
-    for (int k = 0; k < PER; k += 2) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(src + k));
-      acc[k] += w * v.x;
-      acc[k + 1] += w * v.y;
+  float Lp = 0.f;
+  for (long long base = c0; base <= c1; base += 32) {
+    const long long c = base + lane;
+    float wgt = 0.f;
+    if (c <= c1 && cta_start(c, T, P) != cta_start(c + 1, T, P)) {
+      const float2 ml = __ldcg(&p.part_ml[(s + c) * ROWS + r]);
+      wgt = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
+      Lp += wgt * ml.y;
+    }
+    const int cnt = static_cast<int>(c1 - base + 1 < 32 ? c1 - base + 1 : 32);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float wk = __shfl_sync(0xFFFFFFFFu, wgt, k);
+      if (wk != 0.f) {
+        const float* src = p.part_o + ((s + base + k) * ROWS + r) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+          acc[0] += wk * v.x;
+          acc[1] += wk * v.y;
+          acc[2] += wk * v.z;
+          acc[3] += wk * v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+          acc[0] += wk * v.x;
+          acc[1] += wk * v.y;
+        }
+      }
     }
   }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) Lp += __shfl_xor_sync(0xFFFFFFFFu, Lp, m);
+  const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
   const int h = g * p.G + hc * p.Gc + hh;
   __nv_bfloat16* dst = out + ((static_cast<long long>(b) * p.K + i) * p.Hq + h) * D + lane * PER;
 #pragma unroll
@@ -602,13 +688,11 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   p.sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
 
   auto* kfn = attn_splitkv_kernel<D>;
-  if (cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Layout<D>::ALLOC) != cudaSuccess)
-    return ORTHRUS_ECUDA;
+  if (!opt_in_smem(reinterpret_cast<const void*>(kfn), Layout<D>::ALLOC)) return ORTHRUS_ECUDA;
   kfn<<<sms, THREADS, Layout<D>::ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
-  const dim3 cgrid(sh.S, (sh.Gc * sh.K + 7) / 8);
-  attn_combine_kernel<D><<<cgrid, 256, 0, stream>>>(p, sms, static_cast<__nv_bfloat16*>(out));
+  const dim3 cgrid(sh.S, (sh.Gc * sh.K + 3) / 4);
+  attn_combine_kernel<D><<<cgrid, 128, 0, stream>>>(p, sms, static_cast<__nv_bfloat16*>(out));
   if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
   return ORTHRUS_OK;
 }

@@ -44,6 +44,27 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
   return r == CUDA_SUCCESS ? ORTHRUS_OK : ORTHRUS_EINVAL;
 }
 
+bool opt_in_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static const void* done_kernel[64][8] = {};
+  static int done_bytes[64][8] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 8; ++i)
+    if (done_kernel[dev][i] == kernel && done_bytes[dev][i] >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  for (int i = 0; i < 8; ++i)
+    if (done_kernel[dev][i] == nullptr || done_kernel[dev][i] == kernel) {
+      done_kernel[dev][i] = kernel;
+      done_bytes[dev][i] = bytes;
+      break;
+    }
+  return true;
+}
+
 int current_sm_count(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;

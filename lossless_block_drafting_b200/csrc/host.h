@@ -21,6 +21,11 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
 // Number of SMs of the current device (ORTHRUS_ECUDA on failure).
 int current_sm_count(int* sms);
 
+// Raise a kernel's dynamic shared-memory limit on the current device.  Done
+// once per (kernel, device) and remembered, so calls made while a stream is
+// being captured into a CUDA graph issue no attribute call.
+bool opt_in_smem(const void* kernel, int bytes);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }

@@ -58,10 +58,13 @@ inline Plan make_plan(int R) {
   return pl;
 }
 
-__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int32_t* status) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) return;
+    if (globaltimer_ns() - t0 > 200000000ull) {  // 200 ms
+      report(status, ORTHRUS_ETIMEOUT);
+      return;
+    }
   }
 }
 
@@ -186,7 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(sbase + TPR * W_TILE_BYTES, &tmH, full(stage), kc * BK, 0);
       }
     }
-    for (int j = (it > NS ? it - NS : 0); j < it; ++j) mbar_wait_drain(full(j % NS), (j / NS) & 1);
+    for (int j = (it > NS ? it - NS : 0); j < it; ++j) mbar_wait_drain(full(j % NS), (j / NS) & 1, p.dev_status);
   } else if (n_tiles > 0 && warp == 1 && lane == 0) {
     // -------------------------------------------------------- MMA issuer
     const uint32_t idesc = make_idesc_bf16_f32(BM, Npad, false, false);
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (ok) mma_commit(acc_full(buf));
     }
     mma_commit(mma_done);
-    mbar_wait_drain(mma_done, 0);
+    mbar_wait_drain(mma_done, 0, p.dev_status);
   } else if (warp >= 4) {
     // --------------------------------------------------------- epilogue
     const int quarter = warp & 3;
@@ -308,7 +311,7 @@ extern "C" int orthrus_lmhead_workspace_size(int R, int V, size_t* bytes) {
 
 extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H, int V,
                                      int32_t* argmax, float* max_logit, void* workspace,
-                                     size_t ws_bytes, void* stream) {
+                                     size_t ws_bytes, int32_t* dev_status, void* stream) {
   if (h == nullptr || W == nullptr || argmax == nullptr) return ORTHRUS_EINVAL;
   if (R < 0 || V < 1 || H < lmh::BK) return ORTHRUS_EINVAL;
   if (H % lmh::BK != 0) return ORTHRUS_EUNSUPPORTED;
@@ -332,9 +335,7 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     rc = encode_tmap_bf16(&tw16, W, 2, dims, strides, box16);
     if (rc != ORTHRUS_OK) return rc;
   }
-  if (cudaFuncSetAttribute(lmh::lmhead_argmax_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           lmh::SMEM_LIMIT) != cudaSuccess)
+  if (!opt_in_smem(reinterpret_cast<const void*>(lmh::lmhead_argmax_kernel), lmh::SMEM_LIMIT))
     return ORTHRUS_ECUDA;
   const int grid = static_cast<int>((static_cast<long long>(V) + lmh::GROUP - 1) / lmh::GROUP <
                                             sms
@@ -353,7 +354,7 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     if (rc != ORTHRUS_OK) return rc;
     lmh::Params p;
     p.part_keys = keys;
-    p.dev_status = nullptr;
+    p.dev_status = dev_status;
     p.R = Rp;
     p.Npad = pl.Npad;
     p.H = H;

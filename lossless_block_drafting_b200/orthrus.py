@@ -59,7 +59,7 @@ def load(path: str | None = None):
             "orthrus_block_attn_workspace_size": ([I, I, I, I, I, PSZ], I),
             "orthrus_block_attn": ([V, PC, I, I, I, V, V, SZ, V, V], I),
             "orthrus_lmhead_workspace_size": ([I, I, PSZ], I),
-            "orthrus_lmhead_argmax": ([V, V, I, I, I, V, V, V, SZ, V], I),
+            "orthrus_lmhead_argmax": ([V, V, I, I, I, V, V, V, SZ, V, V], I),
             "orthrus_row_argmax_f32": ([V, I, I, V, V], I),
             "orthrus_verify": ([V, V, I, I, V, V, V], I),
             "orthrus_kv_commit": ([PC, V, I, V, V], I),
@@ -154,7 +154,7 @@ def lmhead_workspace_size(R: int, V: int) -> int:
 
 
 def lmhead_argmax(h, W, argmax=None, max_logit=None, workspace=None, stream=None,
-                  want_max: bool = False):
+                  want_max: bool = False, dev_status=None):
     """Greedy token per row of h [R,H] under LM head W [V,H] (bf16) -> int32 [R]."""
     _need(h, torch.bfloat16, "h", 2)
     _need(W, torch.bfloat16, "W", 2)
@@ -171,8 +171,11 @@ def lmhead_argmax(h, W, argmax=None, max_logit=None, workspace=None, stream=None
         _need(max_logit, torch.float32, "max_logit", 1)
     if workspace is None:
         workspace = torch.empty(lmhead_workspace_size(R, V), dtype=torch.uint8, device=h.device)
+    if dev_status is not None:
+        _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_lmhead_argmax(_ptr(h), _ptr(W), R, H, V, _ptr(argmax), _ptr(max_logit),
-                                      _ptr(workspace), workspace.numel(), _stream(stream))
+                                      _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                      _stream(stream))
     _check(rc, "orthrus_lmhead_argmax")
     return (argmax, max_logit) if max_logit is not None else argmax
 

@@ -80,12 +80,12 @@ def test_block_attn_empty_batch_is_a_noop(lib):
 
 def test_lmhead_host_validation(lib):
     f = lib.orthrus_lmhead_argmax
-    assert f(None, A, 4, 128, 10, A, None, A, 1 << 20, None) == ob.EINVAL
-    assert f(A, A, 4, 100, 10, A, None, A, 1 << 20, None) == ob.EUNSUPPORTED  # H % 64
-    assert f(A, A, 4, 32, 10, A, None, A, 1 << 20, None) == ob.EINVAL         # H < 64
-    assert f(A, A, 4, 128, 0, A, None, A, 1 << 20, None) == ob.EINVAL         # V < 1
-    assert f(A + 4, A, 4, 128, 10, A, None, A, 1 << 20, None) == ob.EALIGN
-    assert f(A, A, 0, 128, 10, A, None, A, 1 << 20, None) == ob.OK           # R = 0
+    assert f(None, A, 4, 128, 10, A, None, A, 1 << 20, None, None) == ob.EINVAL
+    assert f(A, A, 4, 100, 10, A, None, A, 1 << 20, None, None) == ob.EUNSUPPORTED  # H % 64
+    assert f(A, A, 4, 32, 10, A, None, A, 1 << 20, None, None) == ob.EINVAL         # H < 64
+    assert f(A, A, 4, 128, 0, A, None, A, 1 << 20, None, None) == ob.EINVAL         # V < 1
+    assert f(A + 4, A, 4, 128, 10, A, None, A, 1 << 20, None, None) == ob.EALIGN
+    assert f(A, A, 0, 128, 10, A, None, A, 1 << 20, None, None) == ob.OK           # R = 0
 
 
 def test_consensus_host_validation(lib):

@@ -22,13 +22,27 @@ ATOL, RTOL_L2, GAP = 2e-2, 5e-3, 1e-3
 
 
 def attn_gpu(case: synth.AttnCase, mode, dev_status=None):
+    """Run the CUDA path; unless the caller inspects the status itself, assert the
+    kernels reported no device-side error (including a bounded wait giving up)."""
     q = case.q.cuda()
     kc = case.k_cache.cuda()
     vc = case.v_cache.cuda()
     cl = torch.from_numpy(case.ctx_lens).cuda()
-    out = ob.block_attn(q, kc, vc, cl, mode, dev_status=dev_status)
+    st = dev_status if dev_status is not None else torch.zeros(1, dtype=torch.int32,
+                                                               device="cuda")
+    out = ob.block_attn(q, kc, vc, cl, mode, dev_status=st)
     torch.cuda.synchronize()
+    if dev_status is None:
+        assert int(st.item()) == 0, ob.status_str(int(st.item()))
     return out.cpu()
+
+
+def lmhead_gpu(h, W, want_max=False):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    res = ob.lmhead_argmax(h.cuda(), W.cuda(), want_max=want_max, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, ob.status_str(int(st.item()))
+    return res
 
 
 def assert_attn_close(got_bf16, ref):
@@ -135,8 +149,7 @@ def _check_argmax(got, ref_am, gap):
 def test_lmhead_argmax_small(R, H, V):
     h, W = synth.lmhead_case(R, H, V, seed=R + V)
     am, top1, gap = oracle.lmhead_argmax(h, W)
-    got, mx = ob.lmhead_argmax(h.cuda(), W.cuda(), want_max=True)
-    torch.cuda.synchronize()
+    got, mx = lmhead_gpu(h, W, want_max=True)
     _check_argmax(got, am, gap)
     np.testing.assert_allclose(mx.cpu().numpy(), top1, rtol=1e-3, atol=1e-3)
 
@@ -145,8 +158,7 @@ def test_lmhead_argmax_two_passes():
     """R > 256 runs in two passes of the kernel."""
     h, W = synth.lmhead_case(300, 128, 5000, seed=3)
     am, _, gap = oracle.lmhead_argmax(h, W)
-    got = ob.lmhead_argmax(h.cuda(), W.cuda())
-    torch.cuda.synchronize()
+    got = lmhead_gpu(h, W)
     _check_argmax(got, am, gap)
 
 
@@ -156,8 +168,7 @@ def test_lmhead_argmax_ties_pick_lowest_index():
     h[:, 0] = 1.0
     W = torch.zeros(V, H, dtype=torch.bfloat16)
     W[[5, 900, 2047], 0] = 3.0          # three-way exact tie for every row
-    got = ob.lmhead_argmax(h.cuda(), W.cuda())
-    torch.cuda.synchronize()
+    got = lmhead_gpu(h, W)
     assert got.cpu().tolist() == [5, 5, 5, 5]
 
 
@@ -165,8 +176,7 @@ def test_lmhead_qwen3_8b_full_vocab():
     """Config-2 LM head: hidden 4096 x vocab 151936, W ~ N(0, 0.02), h ~ N(0, 1)."""
     h, W = synth.lmhead_case(32, 4096, 151936, seed=2)
     am, top1, gap = oracle.lmhead_argmax(h, W)
-    got, mx = ob.lmhead_argmax(h.cuda(), W.cuda(), want_max=True)
-    torch.cuda.synchronize()
+    got, mx = lmhead_gpu(h, W, want_max=True)
     _check_argmax(got, am, gap)
     np.testing.assert_allclose(mx.cpu().numpy(), top1, rtol=1e-3, atol=2e-3)
 
@@ -174,7 +184,7 @@ def test_lmhead_qwen3_8b_full_vocab():
 def test_lmhead_ragged_batch_rows_256_sampled():
     """Config-4 LM head (R = 8 x 32 = 256); the oracle checks 24 sampled rows."""
     h, W = synth.lmhead_case(256, 4096, 151936, seed=9)
-    got = ob.lmhead_argmax(h.cuda(), W.cuda()).cpu().numpy()
+    got = lmhead_gpu(h, W).cpu().numpy()
     rows = np.random.default_rng(0).choice(256, 24, replace=False)
     am, _, gap = oracle.lmhead_argmax(h[rows], W)
     firm = gap >= GAP
