@@ -154,6 +154,31 @@ int orthrus_lmhead_argmax(const void *h, const void *W, int R, int H, int V, int
                           int32_t *dev_status, void *stream);
 
 /*
+ * orthrus_lmhead_argmax for callers that cannot allocate device memory.
+ * (The paper has no counterpart: this is a deployment convenience.)
+ *
+ * Callers such as a plain C host program with no device allocator, a serving
+ * loop whose memory plan is frozen after start-up (cudaMalloc synchronises the
+ * device and may fail under fragmentation), or a runtime that owns all device
+ * memory cannot pass a workspace.  This variant keeps its scratch -- the
+ * per-CTA argmax candidates -- in a fixed 512 KB array inside the library's
+ * own device memory (held on every GPU that loads the library until the
+ * process exits) and otherwise behaves exactly like orthrus_lmhead_argmax.
+ *   - It allocates nothing and calls no allocating routine.
+ *   - The first call on each device looks up the array's device address once;
+ *     make that first call before any stream capture.
+ *   - All calls share the array (it keeps the last call's contents; nothing
+ *     in it has to start zeroed).  Calls that overlap on the GPU race: order
+ *     them on one stream.
+ *   - Returns ORTHRUS_EWORKSPACE, launching nothing, on a device with more
+ *     than 256 SMs (the array's capacity).
+ * Arguments as for orthrus_lmhead_argmax, without the workspace.
+ */
+int orthrus_lmhead_argmax_noalloc(const void *h, const void *W, int R, int H, int V,
+                                  int32_t *argmax, float *max_logit, int32_t *dev_status,
+                                  void *stream);
+
+/*
  * Greedy choice over precomputed fp32 logits (a test helper for verifying
  * from given logits).  logits fp32 [R, V] device -> argmax int32 [R] device
  * (smallest index of the maximum; NaN entries are never chosen).

@@ -22,6 +22,8 @@
 // reach HBM.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "host.h"
 
@@ -369,4 +371,76 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
   }
   return ORTHRUS_OK;
+}
+
+// ---------------------------------------------------------------------------
+// LM head + argmax without any device allocation by the caller.
+//
+// Some callers cannot hand this library a workspace: a plain C or embedded
+// host program that links only this library and has no device allocator of
+// its own, a serving loop whose memory plan is frozen after start-up (where a
+// cudaMalloc could fail under fragmentation or stall every stream, because it
+// synchronises the device), or a runtime that owns all device memory and does
+// not lend scratch to its kernels.  For them this entry point keeps the
+// per-CTA candidate keys in a fixed array in the library's own device memory
+// instead of a caller workspace.
+//
+//   * The array holds at most kNoAllocMaxCtas * 256 keys (512 KB).  It lives in
+//     every GPU that loads the library, for as long as the process runs.
+//   * All calls share it and it keeps the last call's contents.  Nothing in it
+//     needs to start at zero: every CTA overwrites all of its keys before the
+//     reduction reads them.  Calls whose kernels overlap on the GPU (other
+//     streams, other host threads) race on the array; order them on one
+//     stream.
+//   * The first call on each device looks up the array's device address
+//     (cudaGetSymbolAddress) and remembers it.  That query is not a stream
+//     operation; make the first call on a device before any stream capture.
+//   * A device with more SMs than kNoAllocMaxCtas is rejected with
+//     ORTHRUS_EWORKSPACE before anything is launched.
+// The kernels and their arguments are exactly those of orthrus_lmhead_argmax.
+namespace orthrus {
+namespace lmh {
+
+constexpr int kNoAllocMaxCtas = 256;
+static __device__ __align__(256) uint64_t g_noalloc_keys[kNoAllocMaxCtas * MAX_PASS_ROWS];
+
+// Device address of g_noalloc_keys on the current device (looked up once per
+// device; the symbol's host-side name is only a handle, never a pointer the
+// kernel may use).
+int noalloc_scratch(uint64_t** out) {
+  static std::mutex mu;
+  static uint64_t* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ORTHRUS_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_keys) != cudaSuccess || p == nullptr)
+      return ORTHRUS_ECUDA;
+    addr[dev] = static_cast<uint64_t*>(p);
+  }
+  *out = addr[dev];
+  return ORTHRUS_OK;
+}
+
+}  // namespace lmh
+}  // namespace orthrus
+
+extern "C" int orthrus_lmhead_argmax_noalloc(const void* h, const void* W, int R, int H, int V,
+                                             int32_t* argmax, float* max_logit,
+                                             int32_t* dev_status, void* stream) {
+  if (h == nullptr || W == nullptr || argmax == nullptr) return ORTHRUS_EINVAL;
+  if (R < 0 || V < 1 || H < lmh::BK) return ORTHRUS_EINVAL;
+  if (H % lmh::BK != 0) return ORTHRUS_EUNSUPPORTED;
+  if (!aligned16(h) || !aligned16(W)) return ORTHRUS_EALIGN;
+  if (R == 0) return ORTHRUS_OK;
+  int sms = 0;
+  int rc = current_sm_count(&sms);
+  if (rc != ORTHRUS_OK) return rc;
+  if (sms > lmh::kNoAllocMaxCtas) return ORTHRUS_EWORKSPACE;
+  uint64_t* scratch = nullptr;
+  rc = lmh::noalloc_scratch(&scratch);
+  if (rc != ORTHRUS_OK) return rc;
+  return orthrus_lmhead_argmax(h, W, R, H, V, argmax, max_logit, scratch,
+                               sizeof(lmh::g_noalloc_keys), dev_status, stream);
 }

@@ -60,6 +60,7 @@ def load(path: str | None = None):
             "orthrus_block_attn": ([V, PC, I, I, I, V, V, SZ, V, V], I),
             "orthrus_lmhead_workspace_size": ([I, I, PSZ], I),
             "orthrus_lmhead_argmax": ([V, V, I, I, I, V, V, V, SZ, V, V], I),
+            "orthrus_lmhead_argmax_noalloc": ([V, V, I, I, I, V, V, V, V], I),
             "orthrus_row_argmax_f32": ([V, I, I, V, V], I),
             "orthrus_verify": ([V, V, I, I, V, V, V], I),
             "orthrus_kv_commit": ([PC, V, I, V, V], I),
@@ -177,6 +178,33 @@ def lmhead_argmax(h, W, argmax=None, max_logit=None, workspace=None, stream=None
                                       _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                       _stream(stream))
     _check(rc, "orthrus_lmhead_argmax")
+    return (argmax, max_logit) if max_logit is not None else argmax
+
+
+def lmhead_argmax_noalloc(h, W, argmax=None, max_logit=None, stream=None,
+                          want_max: bool = False, dev_status=None):
+    """lmhead_argmax without a caller workspace: the library's own fixed device
+    scratch is used instead (shared by all calls; order overlapping calls on one
+    stream, and make the first call on a device before any graph capture)."""
+    _need(h, torch.bfloat16, "h", 2)
+    _need(W, torch.bfloat16, "W", 2)
+    R, H = h.shape
+    V, H2 = W.shape
+    if H2 != H:
+        raise ValueError("h and W hidden sizes differ")
+    if argmax is None:
+        argmax = torch.empty(R, dtype=torch.int32, device=h.device)
+    _need(argmax, torch.int32, "argmax", 1)
+    if want_max and max_logit is None:
+        max_logit = torch.empty(R, dtype=torch.float32, device=h.device)
+    if max_logit is not None:
+        _need(max_logit, torch.float32, "max_logit", 1)
+    if dev_status is not None:
+        _need(dev_status, torch.int32, "dev_status")
+    rc = load().orthrus_lmhead_argmax_noalloc(_ptr(h), _ptr(W), R, H, V, _ptr(argmax),
+                                              _ptr(max_logit), _ptr(dev_status),
+                                              _stream(stream))
+    _check(rc, "orthrus_lmhead_argmax_noalloc")
     return (argmax, max_logit) if max_logit is not None else argmax
 
 
