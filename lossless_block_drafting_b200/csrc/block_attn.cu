@@ -395,24 +395,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int tile0 = cur.t * TN;
         WARP_WAIT_OR(s_full(w), u & 1, break);
         tc_fence_after();
-        uint32_t ra[32], rb[32];
-        tmem_ld32(t_s, ra);
-        tmem_ld32(t_s + 32, rb);
+        uint32_t sr[TN];
+        tmem_ld64(t_s, sr);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free(w));
 
-        float x[TN];
+        if (tile0 + TN > cur.L + 1) {
+          // Tail tile: some keys lie past some row's limit.  Interior tiles
+          // (every key < L + 1) skip this entirely.
+          const int lim = (r >= rows_valid) ? 0
+                          : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+#pragma unroll
+          for (int c = 0; c < TN; ++c)
+            if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+        }
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < TN; ++c) {
-          const float s = __uint_as_float(c < 32 ? ra[c] : rb[c - 32]);
-          const float v = (tile0 + c < lim) ? s : -INFINITY;
-          x[c] = v;
-          mx4[c & 3] = fmaxf(mx4[c & 3], v);
+        for (int c = 0; c < TN; c += 8) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
+                           __uint_as_float(sr[c + 2 * q + 1]));
         }
-        const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
+        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
         bool waited = false;
         float m_new = m_used;
         if (fresh) {
@@ -439,13 +446,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         m_used = m_new;
         const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-        float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        // p = 2^(s*sl2 - m): scale and shift as packed f32x2 FMAs, exp2 on the
+        // SFU, row sum as packed adds in four independent chains.
+        const float2 sc2 = make_float2(sl2, sl2);
+        const float2 nm2 = make_float2(-m_eff, -m_eff);
+        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+        float x[TN];
 #pragma unroll
-        for (int c = 0; c < TN; ++c) {
-          x[c] = fast_exp2(fmaf(x[c], sl2, -m_eff));
-          rs4[c & 3] += x[c];
+        for (int c = 0; c < TN; c += 2) {
+          const float2 a2 = __ffma2_rn(
+              make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
+          const float2 e2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+          x[c] = e2.x;
+          x[c + 1] = e2.y;
+          acc2[(c >> 1) & 3] = __fadd2_rn(acc2[(c >> 1) & 3], e2);
         }
-        l_sum += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+        const float2 t2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
+        l_sum += t2.x + t2.y;
 
         if (tile0 + TN > kv_end) {
           // The tile runs past the valid keys: zero those V rows so that stale
@@ -587,23 +605,34 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const Params p, int g
       Lp += wgt * ml.y;
     }
     const int cnt = static_cast<int>(c1 - base + 1 < 32 ? c1 - base + 1 : 32);
-#pragma unroll 4
-    for (int k = 0; k < cnt; ++k) {
-      const float wk = __shfl_sync(0xFFFFFFFFu, wgt, k);
-      if (wk != 0.f) {
-        const float* src = p.part_o + ((s + base + k) * ROWS + r) * D + lane * PER;
+    for (int k0 = 0; k0 < cnt; k0 += 8) {
+      // eight independent loads in flight, then the weighted sums
+      float wk[8];
+      float v[8][PER];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        wk[k] = __shfl_sync(0xFFFFFFFFu, wgt, (k0 + k) & 31);
+        const bool live = (k0 + k < cnt) && wk[k] != 0.f;
+        const float* src = p.part_o + ((s + base + k0 + k) * ROWS + r) * D + lane * PER;
         if constexpr (PER == 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-          acc[0] += wk * v.x;
-          acc[1] += wk * v.y;
-          acc[2] += wk * v.z;
-          acc[3] += wk * v.w;
+          const float4 t = live ? __ldcg(reinterpret_cast<const float4*>(src))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
+          v[k][2] = t.z;
+          v[k][3] = t.w;
         } else {
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-          acc[0] += wk * v.x;
-          acc[1] += wk * v.y;
+          const float2 t = live ? __ldcg(reinterpret_cast<const float2*>(src))
+                                : make_float2(0.f, 0.f);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
         }
+        if (!live) wk[k] = 0.f;
       }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += wk[k] * v[k][e];
     }
   }
 #pragma unroll

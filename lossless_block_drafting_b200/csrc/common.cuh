@@ -42,8 +42,16 @@ static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t par
 // reached by part of a warp.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
                                                volatile int* abort_flag, int32_t* status) {
+  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;  // common case
   const bool ok = mbar_wait_bounded(bar, parity, abort_flag, status);
   return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// max(a, b, c) in one instruction (three-input form of max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Monotone map of fp32 onto uint32 (larger float -> larger key); -0 -> +0.
