@@ -175,8 +175,7 @@ class Workload:
         self.ctx_lens = torch.full((B,), L, dtype=torch.int32, device=device)
         self.ctx_init = self.ctx_lens.clone()
         self.attn_out = torch.empty(B, K, Hq, d, dtype=bf, device=device)
-        self.ws_attn = torch.empty(ob.block_attn_workspace_size(B, Hq, Hkv, d, K),
-                                   dtype=torch.uint8, device=device)
+        self.ws_attn = torch.zeros(ob.block_attn_workspace_size(B, Hq, Hkv, d, K), dtype=torch.uint8, device=device)
         self.ws_lm = torch.empty(ob.lmhead_workspace_size(B * K, V), dtype=torch.uint8,
                                  device=device)
         self.draft = torch.empty(B * K, dtype=torch.int32, device=device)

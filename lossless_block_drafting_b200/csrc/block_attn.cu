@@ -15,20 +15,24 @@
 // CTA's contiguous tile range may cross segment boundaries and then emits one
 // partial result per segment piece.  Per CTA (12 warps), each single-thread
 // role on its own ring so no wait of one stream stalls another:
-//   warp 0      TMA: Q tile per piece, K tiles into a 4-stage ring.
-//   warp 2      TMA: V tiles into a 6-stage ring (V is held longer than K);
+//   warp 0      TMA: Q tile per piece, K tile groups into a ring.
+//   warp 2      TMA: V tile groups into a ring;
 //               the whole warp also allocates and frees TMEM.
-//   warp 1      tcgen05 issuer for S = Q K^T into TMEM buffer S_w.
-//   warp 3      tcgen05 issuer for O_w += P V (V read MN-major).
+//   warp 1      tcgen05 issuer for S = Q K^T into TMEM buffer j % 4.
+//   warp 3      tcgen05 issuer for O_w += P V (P from the same TMEM buffer,
+//               V read MN-major from shared memory).
 //   warps 4-11  two softmax warpgroups taking alternate tiles, one thread per
 //               row: S from TMEM, mask, online softmax in the exp2 domain
-//               (rescaling O in TMEM only when the running max grows by more
-//               than 2^8, exact because the final normaliser uses the same
-//               reference), P as bf16 into swizzled shared memory.  At the end
+//               against a running reference max (O in TMEM is rescaled only
+//               when the max grows by more than 2^8, exact because the final
+//               normaliser uses the same reference), P as bf16 back into the
+//               tile's TMEM buffer.  At the end
 //               of a piece group 0 merges both groups' (m, l, O) and writes the
 //               piece's partial result.
-// A second, small kernel merges the partials of each segment by log-sum-exp
-// and writes bf16 output.
+// The kernel is launched cooperatively: after writing its partials every CTA
+// meets the others at a bounded grid barrier and then merges an equal share of
+// the output rows (log-sum-exp over each segment's pieces, bf16 output), so the
+// whole operation is one launch.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -39,28 +43,39 @@
 namespace orthrus {
 namespace attn {
 
-constexpr int TN = 64;        // keys per tile
-constexpr int NK = 4;         // K ring stages (a K tile is released once S = Q K^T is done)
-constexpr int NV = 6;         // V ring stages (a V tile is held until O += P V is done)
+constexpr int TN = 64;        // keys per compute tile
+// K and V are loaded in groups of two consecutive tiles of a segment (one
+// 128-row TMA box per 128-byte column chunk); a tile without a partner (at a
+// segment or CTA-range edge) comes alone in a 64-row box.  Larger boxes keep
+// the TMA engines near HBM bandwidth (measured: 64-row boxes top out at about
+// 80% of it, 128-row boxes near 97%).
 constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
 constexpr int THREADS = 384;  // 12 warps: TMA, MMA, TMEM alloc, spare, 2 softmax groups
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_O = 128;   // O accumulators at 128 and 256 (S buffers at 0 and TN)
+// TMEM columns: two S buffers of 2 * TN fp32 columns, one per load group in
+// flight (S of a group is one N = 128 MMA sequence; tile h of the group owns
+// columns [h * TN, (h + 1) * TN) and its bf16 P overwrites the first TN / 2 of
+// them), then the two softmax groups' O accumulators.
+constexpr int NSB = 2;
+constexpr int SBUF_COLS = 2 * TN;
+constexpr int TMEM_O = NSB * SBUF_COLS;  // O_0 at 256, O_1 at 384
 
 template <int D>
 struct Layout {
   static constexpr int CHUNKS = D / 64;            // 128-byte column chunks of a row
+  static constexpr int NK = D == 128 ? 3 : 6;      // K ring stages (released after S = Q K^T)
+  static constexpr int NV = NK;                    // V ring stages (released after O += P V)
   static constexpr int Q_CHUNK = ROWS * 128;
-  static constexpr int KV_CHUNK = TN * 128;
+  static constexpr int KV_CHUNK = 2 * TN * 128;    // one chunk of a two-tile group
+  static constexpr int HALF = TN * 128;            // offset of the group's second tile
   static constexpr int Q_BYTES = CHUNKS * Q_CHUNK;
   static constexpr int KV_BYTES = CHUNKS * KV_CHUNK;
-  static constexpr int P_BYTES = ROWS * TN * 2;     // one 128-byte chunk per row
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NV * KV_BYTES;
-  static constexpr int OFF_ML = OFF_P + 2 * P_BYTES;   // [ROWS] float2 handed WG1 -> WG0
-  static constexpr int OFF_BAR = OFF_ML + ROWS * 8;
+  static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;  // [ROWS] float2 handed WG1 -> WG0
+  static constexpr int OFF_SCHED = OFF_ML + ROWS * 8;  // 6 x int64 CTA schedule
+  static constexpr int OFF_BAR = OFF_SCHED + 64;
   static constexpr int NBAR = 2 * NK + 2 * NV + 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -71,10 +86,21 @@ struct Params {
   const int32_t* ctx_lens;
   float* part_o;      // [slots][ROWS][D] unnormalised O of each piece
   float2* part_ml;    // [slots][ROWS] (m in log2 units, l)
+  unsigned long long* gbar;  // grid-barrier arrival ticket counter (starts at 0)
+  __nv_bfloat16* out; // [B, K, Hq, D]
   int32_t* dev_status;
   int B, K, Hq, Hkv, G, Gc, nhc, cap, mask_mode;
   float sl2;          // softmax scale * log2(e)
 };
+
+// a * b / c for non-negative operands, with 32-bit division whenever the
+// product and divisor fit (64-bit division is emulated and costly).
+__device__ __forceinline__ long long mul_div(long long a, long long b, long long c) {
+  const unsigned long long prod = static_cast<unsigned long long>(a) * static_cast<unsigned long long>(b);
+  if ((prod >> 32) == 0 && (static_cast<unsigned long long>(c) >> 32) == 0)
+    return static_cast<unsigned int>(prod) / static_cast<unsigned int>(c);
+  return static_cast<long long>(prod / static_cast<unsigned long long>(c));
+}
 
 __device__ __forceinline__ int clamp_len(int L, const Params& p) {
   return L < 0 ? 0 : (L > p.cap - p.K ? p.cap - p.K : L);
@@ -104,8 +130,8 @@ __device__ void cursor_seek(Cursor& c, const Params& p, long long x) {
     cursor_load(c, p);
   }
   const long long local = x - c.base;
-  c.seg = static_cast<int>(local / c.nt);
-  c.t = static_cast<int>(local % c.nt);
+  c.seg = static_cast<int>(mul_div(local, 1, c.nt));
+  c.t = static_cast<int>(local - static_cast<long long>(c.seg) * c.nt);
 }
 
 __device__ __forceinline__ void cursor_next(Cursor& c, const Params& p) {
@@ -129,13 +155,83 @@ __device__ long long total_tiles(const Params& p, bool report_errors) {
   return T;
 }
 
+// Load groups: a group starts at an even tile of a segment (or at the CTA's
+// first tile) and ends at an odd tile, the segment's last tile or the CTA's
+// last tile.  Every role derives the same groups from the same cursor.
+__device__ __forceinline__ bool group_first(const Cursor& c, int j) {
+  return j == 0 || (c.t & 1) == 0;
+}
+__device__ __forceinline__ bool group_last(const Cursor& c, int j, int n) {
+  return j == n - 1 || (c.t & 1) == 1 || c.t + 1 == c.nt;
+}
+
+// Work partition over P CTAs.  When the segments fit (S <= P), every CTA
+// works inside a single segment: segment s gets 1 + floor((P - S) * n_s / T)
+// CTAs (the first P - sum of those segments get one more) and splits its n_s
+// tiles evenly among them, so no CTA pays for a mid-range piece boundary
+// (pipeline drain, partial write, Q reload).  With more segments than CTAs
+// the flat tile range is split evenly (stream-K style) and a CTA may cross
+// segments.  Both kernels derive the same partition from ctx_lens.
+struct SegWalk {
+  int b, seg, ns;       // current segment (sequence b, KV head x head chunk seg), its tiles
+  long long Ts;         // first flat tile of the segment
+  int c0, cn;           // its CTAs [c0, c0 + cn)
+};
+
+template <typename F>
+__device__ __forceinline__ void walk_segments(const Params& p, long long T, int P, F&& f) {
+  const int nseg = p.Hkv * p.nhc;
+  const long long S = static_cast<long long>(p.B) * nseg;
+  long long sum_c = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int ns = n_tiles(clamp_len(__ldg(p.ctx_lens + b), p), p);
+    const long long extra = mul_div(static_cast<long long>(P) - S, ns, T);
+    for (int sg = 0; sg < nseg; ++sg) sum_c += 1 + extra;
+  }
+  const long long rem = P - sum_c;  // < S
+  long long Ts = 0, c0 = 0, si = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const int ns = n_tiles(clamp_len(__ldg(p.ctx_lens + b), p), p);
+    const long long extra = mul_div(static_cast<long long>(P) - S, ns, T);
+    for (int sg = 0; sg < nseg; ++sg, ++si) {
+      const int cn = static_cast<int>(1 + extra + (si < rem ? 1 : 0));
+      SegWalk w{b, sg, ns, Ts, static_cast<int>(c0), cn};
+      if (f(w)) return;
+      Ts += ns;
+      c0 += cn;
+    }
+  }
+}
+
+__device__ __forceinline__ bool segment_partition(const Params& p, int P) {
+  return static_cast<long long>(p.B) * p.Hkv * p.nhc <= P;
+}
+
 // First tile of CTA c when T tiles are split over P CTAs.
 __device__ __forceinline__ long long cta_start(long long c, long long T, long long P) {
-  return c * T / P;
+  return mul_div(c, T, P);
 }
 // The CTA whose range contains tile x (the last c with cta_start(c) <= x).
 __device__ __forceinline__ long long cta_of(long long x, long long T, long long P) {
-  return ((x + 1) * P - 1) / T;
+  return mul_div((x + 1) * P - 1, 1, T);
+}
+
+// Flat tile range [x0, x1) of CTA c.
+__device__ void cta_range(const Params& p, long long T, int P, int c, long long* x0,
+                          long long* x1) {
+  if (!segment_partition(p, P)) {
+    *x0 = cta_start(c, T, P);
+    *x1 = cta_start(c + 1, T, P);
+    return;
+  }
+  *x0 = *x1 = T;
+  walk_segments(p, T, P, [&](const SegWalk& w) {
+    if (c < w.c0 || c >= w.c0 + w.cn) return false;
+    const long long k = c - w.c0;
+    *x0 = w.Ts + mul_div(k, w.ns, w.cn);
+    *x1 = w.Ts + mul_div(k + 1, w.ns, w.cn);
+    return true;
+  });
 }
 
 // Wait that ignores the abort flag, used only to drain in-flight async work
@@ -150,12 +246,192 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
   }
 }
 
+// Grid-wide barrier of a cooperative launch (all CTAs resident), split into
+// arrive and wait so a CTA can do independent work in between.  Thread 0 of
+// each CTA takes a ticket from a 64-bit counter that only ever grows by
+// nctas per launch (so it stays a multiple of nctas between launches and
+// never needs resetting); the generation is complete once the counter reaches
+// the next multiple.  Bounded: a wait that gives up reports ETIMEOUT.
+__device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* gbar,
+                                                          unsigned int nctas) {
+  __threadfence();
+  const unsigned long long ticket = atomicAdd(gbar, 1ull);
+  return (ticket / nctas + 1) * nctas;
+}
+
+__device__ void grid_wait(unsigned long long* gbar, unsigned long long target,
+                          int32_t* status) {
+  volatile unsigned long long* v = gbar;
+  const uint64_t t0 = globaltimer_ns();
+  while (*v < target) {
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      report(status, ORTHRUS_ETIMEOUT);
+      break;
+    }
+    __nanosleep(32);
+  }
+  __threadfence();
+}
+
+// CTAs [*c0, *c1] may hold pieces of segment s = (b, seg); *tall is the flat
+// tile total in stream-K mode or -1 under the per-segment partition.
+__device__ void segment_ctas(const Params& p, int P, int b, int seg, long long* c0,
+                             long long* c1, long long* tall, int* ntb) {
+  const int nseg = p.Hkv * p.nhc;
+  long long T = 0, Ts = 0;
+  int nt_b = 1;
+  for (int bb = 0; bb < p.B; ++bb) {
+    const int nt = n_tiles(clamp_len(__ldg(p.ctx_lens + bb), p), p);
+    if (bb == b) {
+      Ts = T + static_cast<long long>(seg) * nt;
+      nt_b = nt;
+    }
+    T += static_cast<long long>(nseg) * nt;
+  }
+  *ntb = nt_b;
+  if (segment_partition(p, P)) {
+    *c0 = 0;
+    *c1 = -1;
+    walk_segments(p, T, P, [&](const SegWalk& w) {
+      if (w.b != b || w.seg != seg) return false;
+      *c0 = w.c0;
+      *c1 = w.c0 + w.cn - 1;
+      return true;
+    });
+    *tall = -1;
+  } else {
+    *c0 = cta_of(Ts, T, P);
+    *c1 = cta_of(Ts + nt_b - 1, T, P);
+    *tall = T;
+  }
+}
+
+// Pieces of one segment, as seen by the merge: CTAs [c0, c1]; when `dense`
+// every one of them wrote a piece, otherwise empty CTAs are skipped (tall is
+// the flat tile total in stream-K mode or -1 under the per-segment partition).
+struct SegPieces {
+  long long c0, c1, tall;
+  int ntb, dense;
+};
+
+__device__ SegPieces segment_pieces(const Params& p, int P, long long s) {
+  const int nseg = p.Hkv * p.nhc;
+  SegPieces sp;
+  segment_ctas(p, P, static_cast<int>(s / nseg), static_cast<int>(s % nseg), &sp.c0, &sp.c1,
+               &sp.tall, &sp.ntb);
+  if (sp.tall >= 0)
+    sp.dense = sp.tall >= P;                    // stream-K: no empty CTA at all
+  else
+    sp.dense = (sp.c1 - sp.c0 + 1) <= sp.ntb;  // no more CTAs than tiles
+  return sp;
+}
+
+constexpr int MERGE_SEGS = 64;  // segment records precomputed per CTA
+
+// Merge the pieces of output rows [r0, r1) (flat over segments x rows of a
+// segment) by log-sum-exp; one warp per row, lane owns D/32 columns, twelve
+// pieces' loads in flight per round.  Segment records for the CTA's rows are
+// in `segs` (first segment s_first, n_segs of them); rows beyond them fall
+// back to computing the record in lane 0.
+template <int D>
+__device__ void merge_rows(const Params& p, int P, long long r0, long long r1, int warp,
+                           int nwarps, int lane, const SegPieces* segs, long long s_first,
+                           int n_segs) {
+  constexpr int PER = D / 32;
+  constexpr int BATCH = 12;
+  const int nseg = p.Hkv * p.nhc;
+  const int RV = p.Gc * p.K;
+  for (long long q = r0 + warp; q < r1; q += nwarps) {
+    const long long s = mul_div(q, 1, RV);
+    const int r = static_cast<int>(q - s * RV);
+    const int b = static_cast<int>(s / nseg), seg = static_cast<int>(s % nseg);
+    const int g = seg / p.nhc, hc = seg % p.nhc;
+    const int i = r / p.Gc, hh = r % p.Gc;
+    if (hc * p.Gc + hh >= p.G) continue;
+    SegPieces sp;
+    if (s - s_first < n_segs) {
+      sp = segs[s - s_first];
+    } else {
+      SegPieces t{};
+      if (lane == 0) t = segment_pieces(p, P, s);
+      sp.c0 = __shfl_sync(0xFFFFFFFFu, t.c0, 0);
+      sp.c1 = __shfl_sync(0xFFFFFFFFu, t.c1, 0);
+      sp.tall = __shfl_sync(0xFFFFFFFFu, t.tall, 0);
+      sp.ntb = __shfl_sync(0xFFFFFFFFu, t.ntb, 0);
+      sp.dense = __shfl_sync(0xFFFFFFFFu, t.dense, 0);
+    }
+    auto has_piece = [&](long long c) {
+      if (sp.dense) return true;
+      if (sp.tall >= 0) return cta_start(c, sp.tall, P) != cta_start(c + 1, sp.tall, P);
+      const long long k = c - sp.c0, cn = sp.c1 - sp.c0 + 1;
+      return mul_div(k, sp.ntb, cn) != mul_div(k + 1, sp.ntb, cn);
+    };
+    float m = -INFINITY, l = 0.f;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    for (long long base = sp.c0; base <= sp.c1; base += BATCH) {
+      float2 ml[BATCH];
+      float v[BATCH][PER];
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) {
+        const long long c = base + k;
+        const bool live = c <= sp.c1 && has_piece(c);
+        ml[k] = live ? __ldcg(&p.part_ml[(s + c) * ROWS + r]) : make_float2(-INFINITY, 0.f);
+        const float* src = p.part_o + ((s + c) * ROWS + r) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 t = live ? __ldcg(reinterpret_cast<const float4*>(src))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
+          v[k][2] = t.z;
+          v[k][3] = t.w;
+        } else {
+          const float2 t = live ? __ldcg(reinterpret_cast<const float2*>(src))
+                                : make_float2(0.f, 0.f);
+          v[k][0] = t.x;
+          v[k][1] = t.y;
+        }
+      }
+      float mr = m;
+#pragma unroll
+      for (int k = 0; k < BATCH; ++k) mr = fmaxf(mr, ml[k].x);
+      if (mr != -INFINITY) {
+        const float a = (m == -INFINITY) ? 0.f : fast_exp2(m - mr);
+        l *= a;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] *= a;
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+          const float wk = (ml[k].x == -INFINITY) ? 0.f : fast_exp2(ml[k].x - mr);
+          l += wk * ml[k].y;
+#pragma unroll
+          for (int e = 0; e < PER; ++e) acc[e] += wk * v[k][e];
+        }
+        m = mr;
+      }
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const int h = g * p.G + hc * p.Gc + hh;
+    __nv_bfloat16* dst =
+        p.out + ((static_cast<long long>(b) * p.K + i) * p.Hq + h) * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; e += 2)
+      *reinterpret_cast<__nv_bfloat162*>(dst + e) =
+          __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_splitkv_kernel(const __grid_constant__ CUtensorMap tmQ,
-                        const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const Params p) {
+                        const __grid_constant__ CUtensorMap tmK2,
+                        const __grid_constant__ CUtensorMap tmK1,
+                        const __grid_constant__ CUtensorMap tmV2,
+                        const __grid_constant__ CUtensorMap tmV1, const Params p) {
   using Ly = Layout<D>;
+  constexpr int NK = Ly::NK;
+  constexpr int NV = Ly::NV;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
@@ -173,10 +449,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t bar2 = bar + 8u * (2 * NK + 2 * NV);
   const uint32_t q_full = bar2;
   const uint32_t q_empty = bar2 + 8u;
-  auto s_full = [&](int i) { return bar2 + 8u * (2 + i); };
-  auto s_free = [&](int i) { return bar2 + 8u * (4 + i); };
-  auto p_full = [&](int i) { return bar2 + 8u * (6 + i); };
-  auto p_empty = [&](int i) { return bar2 + 8u * (8 + i); };
+  auto s_full = [&](int i) { return bar2 + 8u * (2 + i); };   // S of buffer i ready
+  auto sb_free = [&](int i) { return bar2 + 8u * (4 + i); };  // P*V done with buffer i
+  auto p_full = [&](int i) { return bar2 + 8u * (6 + i); };   // P of buffer i / 2, half i & 1
   const uint32_t o_full = bar2 + 8u * 10;
   const uint32_t o_free = bar2 + 8u * 11;
   const uint32_t mma_done = bar2 + 8u * 12;  // both MMA issuers commit once at exit
@@ -184,11 +459,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
   float2* ml_xchg = reinterpret_cast<float2*>(smem + Ly::OFF_ML);
 
-  const long long T = total_tiles(p, blockIdx.x == 0 && threadIdx.x == 0);
-  const long long Pc = gridDim.x;
-  const long long x0 = cta_start(blockIdx.x, T, Pc);
-  const long long x1 = cta_start(blockIdx.x + 1, T, Pc);
-  const int n = static_cast<int>(x1 - x0);
+  // The CTA's tile range and its starting cursor are computed once, by
+  // thread 0, and shared.
+  long long* sched = reinterpret_cast<long long*>(smem + Ly::OFF_SCHED);
+  if (threadIdx.x == 0) {
+    const long long T = total_tiles(p, blockIdx.x == 0);
+    long long a, b;
+    cta_range(p, T, gridDim.x, blockIdx.x, &a, &b);
+    Cursor c0{};
+    if (b > a) cursor_seek(c0, p, a);
+    sched[0] = a;
+    sched[1] = b;
+    sched[2] = c0.base;
+    sched[3] = (static_cast<long long>(c0.b) << 32) | static_cast<unsigned int>(c0.seg);
+    sched[4] = (static_cast<long long>(c0.t) << 32) | static_cast<unsigned int>(c0.L);
+    sched[5] = c0.nt;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -201,11 +487,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSB; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 4);
-      mbar_init(p_full(i), 4);
-      mbar_init(p_empty(i), 1);
+      mbar_init(sb_free(i), 1);
+      mbar_init(p_full(2 * i), 4);
+      mbar_init(p_full(2 * i + 1), 4);
     }
     mbar_init(o_full, 1);
     mbar_init(o_free, 4);
@@ -221,6 +507,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const long long x0 = sched[0];
+  const int n = static_cast<int>(sched[1] - sched[0]);
+  Cursor start;
+  start.base = sched[2];
+  start.b = static_cast<int>(sched[3] >> 32);
+  start.seg = static_cast<int>(sched[3] & 0xffffffff);
+  start.t = static_cast<int>(sched[4] >> 32);
+  start.L = static_cast<int>(sched[4] & 0xffffffff);
+  start.nt = static_cast<int>(sched[5]);
   const int nseg = p.Hkv * p.nhc;
 
 #define WAIT_OR(barrier, parity, on_fail) \
@@ -231,11 +526,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (n > 0 && warp == 0 && lane == 0) {
     // ------------------------------------------------- Q and K producer
     prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmK2);
+    prefetch_tmap(&tmK1);
     const uint64_t policy = policy_evict_first();
     Cursor cur;
-    cursor_seek(cur, p, x0);
-    int pieces = 0, issued = 0;
+    cur = start;
+    int pieces = 0, gi = 0;
     const uint32_t q_tx = static_cast<uint32_t>(p.Gc * p.K * D * 2);
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cur.t == 0;
@@ -248,48 +544,66 @@ __global__ void __launch_bounds__(THREADS, 1)
                       g * p.G + hc * p.Gc, cur.b * p.K);
         ++pieces;
       }
-      const int stage = j % NK;
-      const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
-      WAIT_OR(empty_k(stage), ((j / NK) & 1) ^ 1, break);
-      mbar_arrive_expect_tx(full_k(stage), Ly::KV_BYTES);
-      for (int c = 0; c < Ly::CHUNKS; ++c)
-        tma_load_2d_hint(sb0 + Ly::OFF_K + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK, &tmK,
-                         full_k(stage), c * 64, row0, policy);
-      ++issued;
+      if (group_first(cur, j)) {
+        const bool pair = !group_last(cur, j, n);
+        const int stage = gi % NK;
+        const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
+        WAIT_OR(empty_k(stage), ((gi / NK) & 1) ^ 1, break);
+        mbar_arrive_expect_tx(full_k(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
+        for (int c = 0; c < Ly::CHUNKS; ++c)
+          tma_load_2d_hint(sb0 + Ly::OFF_K + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
+                           pair ? &tmK2 : &tmK1, full_k(stage), c * 64, row0, policy);
+        ++gi;
+      }
       cursor_next(cur, p);
     }
     // Drain: every issued copy must have landed before the CTA may exit.
-    for (int j = (issued > NK ? issued - NK : 0); j < issued; ++j)
-      mbar_wait_drain(full_k(j % NK), (j / NK) & 1, p.dev_status);
+    for (int q = (gi > NK ? gi - NK : 0); q < gi; ++q)
+      mbar_wait_drain(full_k(q % NK), (q / NK) & 1, p.dev_status);
     if (pieces > 0) mbar_wait_drain(q_full, (pieces - 1) & 1, p.dev_status);
   } else if (n > 0 && warp == 2 && lane == 0) {
     // ------------------------------------------------------- V producer
-    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmV2);
+    prefetch_tmap(&tmV1);
     const uint64_t policy = policy_evict_first();
     Cursor cur;
-    cursor_seek(cur, p, x0);
-    int issued = 0;
+    cur = start;
+    int gi = 0;
     for (int j = 0; j < n; ++j) {
-      const int g = cur.seg / p.nhc;
-      const int stage = j % NV;
-      const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
-      WAIT_OR(empty_v(stage), ((j / NV) & 1) ^ 1, break);
-      mbar_arrive_expect_tx(full_v(stage), Ly::KV_BYTES);
-      for (int c = 0; c < Ly::CHUNKS; ++c)
-        tma_load_2d_hint(sb0 + Ly::OFF_V + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK, &tmV,
-                         full_v(stage), c * 64, row0, policy);
-      ++issued;
+      if (group_first(cur, j)) {
+        const bool pair = !group_last(cur, j, n);
+        const int g = cur.seg / p.nhc;
+        const int stage = gi % NV;
+        const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
+        WAIT_OR(empty_v(stage), ((gi / NV) & 1) ^ 1, break);
+        mbar_arrive_expect_tx(full_v(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
+        for (int c = 0; c < Ly::CHUNKS; ++c)
+          tma_load_2d_hint(sb0 + Ly::OFF_V + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
+                           pair ? &tmV2 : &tmV1, full_v(stage), c * 64, row0, policy);
+        ++gi;
+      }
       cursor_next(cur, p);
     }
-    for (int j = (issued > NV ? issued - NV : 0); j < issued; ++j)
-      mbar_wait_drain(full_v(j % NV), (j / NV) & 1, p.dev_status);
+    for (int q = (gi > NV ? gi - NV : 0); q < gi; ++q)
+      mbar_wait_drain(full_v(q % NV), (q / NV) & 1, p.dev_status);
   } else if (n > 0 && warp == 1 && lane == 0) {
     // ------------------------------------------------ S = Q K^T issuer
-    // Tile j belongs to softmax warpgroup w = j & 1 and lands in TMEM S_w.
-    const uint32_t id_s = make_idesc_bf16_f32(ROWS, TN, false, false);
+    // One N = 128 (or 64 for a lone tile) MMA sequence per load group into
+    // TMEM buffer g % 2; the buffer is reused once P*V of group g - 2 is done.
+    // Descriptors are built once; per group only the stage offset is added.
+    const uint32_t id_s2 = make_idesc_bf16_f32(ROWS, 2 * TN, false, false);
+    const uint32_t id_s1 = make_idesc_bf16_f32(ROWS, TN, false, false);
+    uint64_t qd[D / 16], kd[D / 16];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qd[kk] = make_sdesc(sb0 + Ly::OFF_Q + (kk >> 2) * Ly::Q_CHUNK + (kk & 3) * 32, 16, 1024,
+                          kSwizzle128B);
+      kd[kk] = make_sdesc(sb0 + Ly::OFF_K + (kk >> 2) * Ly::KV_CHUNK + (kk & 3) * 32, 16, 1024,
+                          kSwizzle128B);
+    }
     Cursor cs;
-    cursor_seek(cs, p, x0);
-    int q_seen = 0;
+    cs = start;
+    int q_seen = 0, gi = 0;
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cs.t == 0;
       const bool last = (j == n - 1) || cs.t == cs.nt - 1;
@@ -297,27 +611,26 @@ __global__ void __launch_bounds__(THREADS, 1)
         WAIT_OR(q_full, q_seen & 1, break);
         ++q_seen;
       }
-      const int stage = j % NK;
-      WAIT_OR(full_k(stage), (j / NK) & 1, break);
-      const int w = j & 1;
-      const int u = j >> 1;
-      if (u >= 1) {
-        WAIT_OR(s_free(w), (u - 1) & 1, break);
-      }
-      tc_fence_after();
-      const uint32_t qa = sb0 + Ly::OFF_Q;
-      const uint32_t ka = sb0 + Ly::OFF_K + stage * Ly::KV_BYTES;
+      const bool glast = group_last(cs, j, n);
+      if (group_first(cs, j)) {
+        const int stage = gi % NK;
+        const int gb = gi & 1;
+        WAIT_OR(full_k(stage), (gi / NK) & 1, break);
+        if (gi >= NSB) {
+          WAIT_OR(sb_free(gb), ((gi >> 1) - 1) & 1, break);
+        }
+        tc_fence_after();
+        const uint64_t koff = static_cast<uint64_t>((stage * Ly::KV_BYTES) >> 4);
+        const uint32_t id = glast ? id_s1 : id_s2;
+        const uint32_t dst = tmem + gb * SBUF_COLS;
+        mma_bf16_ss(dst, qd[0], kd[0] + koff, id, 0u);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t ad = make_sdesc(qa + (kk >> 2) * Ly::Q_CHUNK + (kk & 3) * 32, 16, 1024,
-                                       kSwizzle128B);
-        const uint64_t bd = make_sdesc(ka + (kk >> 2) * Ly::KV_CHUNK + (kk & 3) * 32, 16, 1024,
-                                       kSwizzle128B);
-        mma_bf16_ss(tmem + w * TN, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < D / 16; ++kk) mma_bf16_ss(dst, qd[kk], kd[kk] + koff, id, 1u);
+        mma_commit(empty_k(stage));
+        mma_commit(s_full(gb));
       }
-      mma_commit(empty_k(stage));
-      mma_commit(s_full(w));
       if (last) mma_commit(q_empty);
+      if (glast) ++gi;
       cursor_next(cs, p);
     }
     // every MMA of both issuers must be complete before TMEM is released
@@ -326,9 +639,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (n > 0 && warp == 3 && lane == 0) {
     // ------------------------------------------------ O_w += P V issuer
     const uint32_t id_pv = make_idesc_bf16_f32(ROWS, D, false, true);
+    uint64_t vd[TN / 16];
+#pragma unroll
+    for (int kk = 0; kk < TN / 16; ++kk)
+      // V is [keys x d] with d contiguous: MN-major B operand; 16 keys per step
+      // = two 8-row swizzle atoms (2048 B); d chunks Ly::KV_CHUNK apart.
+      vd[kk] = make_sdesc(sb0 + Ly::OFF_V + kk * 2048, Ly::KV_CHUNK, 1024, kSwizzle128B);
     Cursor cp;
-    cursor_seek(cp, p, x0);
-    int pieces_done = 0, jp = 0;
+    cp = start;
+    int pieces_done = 0, jp = 0, gi = 0;
+    int pf_uses[2 * NSB] = {0, 0, 0, 0};  // completed phases seen per P barrier
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cp.t == 0;
       const bool last = (j == n - 1) || cp.t == cp.nt - 1;
@@ -339,23 +659,28 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
       const int w = j & 1;
-      WAIT_OR(p_full(w), (j >> 1) & 1, break);
-      const int stage = j % NV;
-      WAIT_OR(full_v(stage), (j / NV) & 1, break);
-      tc_fence_after();
-      const uint32_t pa = sb0 + Ly::OFF_P + w * Ly::P_BYTES;
-      const uint32_t va = sb0 + Ly::OFF_V + stage * Ly::KV_BYTES;
-      const bool fresh = (j - jp) < 2;  // first tile of group w in this piece
-#pragma unroll
-      for (int kk = 0; kk < TN / 16; ++kk) {
-        const uint64_t ad = make_sdesc(pa + kk * 32, 16, 1024, kSwizzle128B);
-        // V is [keys x d] with d contiguous: MN-major B operand.  16 keys per
-        // step = two 8-row swizzle atoms (2048 B); d chunks Ly::KV_CHUNK apart.
-        const uint64_t bd = make_sdesc(va + kk * 2048, Ly::KV_CHUNK, 1024, kSwizzle128B);
-        mma_bf16_ss(tmem + TMEM_O + w * 128, ad, bd, id_pv, (fresh && kk == 0) ? 0u : 1u);
+      const bool gfirst = group_first(cp, j), glast = group_last(cp, j, n);
+      const int gb = gi & 1, half = gfirst ? 0 : 1;
+      const int pb = 2 * gb + half;
+      WAIT_OR(p_full(pb), pf_uses[pb] & 1, break);
+      ++pf_uses[pb];
+      const int stage = gi % NV;
+      if (gfirst) {
+        WAIT_OR(full_v(stage), (gi / NV) & 1, break);
       }
-      mma_commit(empty_v(stage));
-      mma_commit(p_empty(w));
+      tc_fence_after();
+      const uint64_t voff = static_cast<uint64_t>((stage * Ly::KV_BYTES + half * Ly::HALF) >> 4);
+      const uint32_t a_p = tmem + gb * SBUF_COLS + half * TN;  // P: 16 keys = 8 columns
+      const uint32_t dst = tmem + TMEM_O + w * 128;
+      const bool fresh = (j - jp) < 2;  // first tile of group w in this piece
+      mma_bf16_ts(dst, a_p, vd[0] + voff, id_pv, fresh ? 0u : 1u);
+#pragma unroll
+      for (int kk = 1; kk < TN / 16; ++kk) mma_bf16_ts(dst, a_p + kk * 8, vd[kk] + voff, id_pv, 1u);
+      if (glast) {
+        mma_commit(empty_v(stage));
+        mma_commit(sb_free(gb));
+        ++gi;
+      }
       if (last) {
         mma_commit(o_full);
         ++pieces_done;
@@ -369,14 +694,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int w = (warp - 4) >> 2;            // softmax warpgroup: even / odd tiles
     const int r = (warp & 3) * 32 + lane;     // query row == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t t_s = lane_base + w * TN;
     const uint32_t t_o = lane_base + TMEM_O + w * 128;
     const int rows_valid = p.Gc * p.K;
     const int i_row = r / p.Gc;
     const float sl2 = p.sl2;
     Cursor cur;
-    cursor_seek(cur, p, x0);
-    int pieces = 0, jp = 0;
+    cur = start;
+    int pieces = 0, jp = 0, gi = 0, prev_gi = 0;
     float m_used = -INFINITY, l_sum = 0.f;
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cur.t == 0;
@@ -388,19 +712,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if ((j & 1) == w) {
         const bool fresh = (j - jp) < 2;
-        const int u = j >> 1;
+        const int gb = gi & 1;
+        const int half = group_first(cur, j) ? 0 : 1;
+        const uint32_t t_s = lane_base + gb * SBUF_COLS + half * TN;
         const int kv_end = cur.L + p.K;
-        const int lim = (r >= rows_valid) ? 0
-                        : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
         const int tile0 = cur.t * TN;
-        WARP_WAIT_OR(s_full(w), u & 1, break);
+        WARP_WAIT_OR(s_full(gb), (gi >> 1) & 1, break);
         tc_fence_after();
         uint32_t sr[TN];
         tmem_ld64(t_s, sr);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free(w));
 
         if (tile0 + TN > cur.L + 1) {
           // Tail tile: some keys lie past some row's limit.  Interior tiles
@@ -411,56 +732,81 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < TN; ++c)
             if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < TN; c += 8) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
-                           __uint_as_float(sr[c + 2 * q + 1]));
-        }
-        const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
-        bool waited = false;
-        float m_new = m_used;
-        if (fresh) {
-          m_new = mx;
-        } else if (__any_sync(0xFFFFFFFFu, mx > m_used + 8.f)) {
-          m_new = fmaxf(m_used, mx);
-          const float f = (m_new == -INFINITY) ? 1.f
-                          : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
-          // O_w may only be touched once this group's previous P*V completed.
-          WARP_WAIT_OR(p_empty(w), (u - 1) & 1, break);
-          waited = true;
-          tc_fence_after();
-#pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(t_o + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-            tmem_st32(t_o + c0, o);
-          }
-          tmem_wait_st();
-          l_sum *= f;
-        }
-        m_used = m_new;
-        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-        // p = 2^(s*sl2 - m): scale and shift as packed f32x2 FMAs, exp2 on the
-        // SFU, row sum as packed adds in four independent chains.
+        // p = 2^(s*sl2 - m) against the running reference m (scale and shift as
+        // packed f32x2 FMAs, exp2 on the SFU, row sum as packed adds); the
+        // tile max is computed alongside and only a jump of the max by more
+        // than 2^8 forces the slow path that rescales O and redoes the tile.
+        // The first tile of a piece takes its own max first.
         const float2 sc2 = make_float2(sl2, sl2);
-        const float2 nm2 = make_float2(-m_eff, -m_eff);
-        float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                          make_float2(0.f, 0.f)};
         float x[TN];
+        float2 acc2[4];
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        // exps against m_ref, also folding the tile max when want_max (each S
+        // value is read once, so S and P are never both live in registers)
+        auto exps = [&](float m_ref, bool want_max) {
+          const float m_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
+          const float2 nm2 = make_float2(-m_eff, -m_eff);
 #pragma unroll
-        for (int c = 0; c < TN; c += 2) {
-          const float2 a2 = __ffma2_rn(
-              make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
-          const float2 e2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-          x[c] = e2.x;
-          x[c + 1] = e2.y;
-          acc2[(c >> 1) & 3] = __fadd2_rn(acc2[(c >> 1) & 3], e2);
+          for (int q = 0; q < 4; ++q) acc2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < TN; c += 2) {
+            const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
+            if (want_max) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], s0, s1);
+            const float2 a2 = __ffma2_rn(make_float2(s0, s1), sc2, nm2);
+            const float2 e2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+            x[c] = e2.x;
+            x[c + 1] = e2.y;
+            acc2[(c >> 1) & 3] = __fadd2_rn(acc2[(c >> 1) & 3], e2);
+          }
+        };
+        auto reduce_max = [&]() {
+          return fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
+        };
+        if (fresh) {
+#pragma unroll
+          for (int c = 0; c < TN; c += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
+                             __uint_as_float(sr[c + 2 * q + 1]));
+          }
+          m_used = reduce_max();
+          exps(m_used, false);
+        } else {
+          exps(m_used, true);
+          const float mx = reduce_max();
+          if (__any_sync(0xFFFFFFFFu, mx > m_used + 8.f)) {
+            const float m_new = fmaxf(m_used, mx);
+            const float f = (m_new == -INFINITY) ? 1.f
+                            : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
+            // O_w may only be touched once this group's previous P*V (tile
+            // j - 2, in load group prev_gi) has completed.
+            WARP_WAIT_OR(sb_free(prev_gi & 1), (prev_gi >> 1) & 1, break);
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(t_o + c0, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+              tmem_st32(t_o + c0, o);
+            }
+            tmem_wait_st();
+            l_sum *= f;
+            m_used = m_new;
+            // S is still in its TMEM buffer: reload it (re-masked) and redo
+            tmem_ld64(t_s, sr);
+            tmem_wait_ld();
+            if (tile0 + TN > cur.L + 1) {
+              const int lim = (r >= rows_valid) ? 0
+                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+#pragma unroll
+              for (int c = 0; c < TN; ++c)
+                if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+            }
+            exps(m_used, false);
+          }
         }
         const float2 t2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
         l_sum += t2.x + t2.y;
@@ -468,11 +814,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (tile0 + TN > kv_end) {
           // The tile runs past the valid keys: zero those V rows so that stale
           // or NaN cache contents cannot reach O through 0 * NaN.
-          const int stage = j % NV;
-          WARP_WAIT_OR(full_v(stage), (j / NV) & 1, break);
+          const int stage = gi % NV;
+          WARP_WAIT_OR(full_v(stage), (gi / NV) & 1, break);
           const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
           const int per_chunk = (TN - nv) * 8;
-          uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES;
+          uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES +
+                        (group_first(cur, j) ? 0 : Ly::HALF);
           for (int q = r; q < per_chunk * Ly::CHUNKS; q += ROWS) {
             const int ch = q / per_chunk, rem = q % per_chunk;
             *reinterpret_cast<uint4*>(vt + ch * Ly::KV_CHUNK + (nv + rem / 8) * 128 +
@@ -480,22 +827,15 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           fence_proxy_async_smem();
         }
-        if (u >= 1 && !waited) {
-          WARP_WAIT_OR(p_empty(w), (u - 1) & 1, break);
-        }
-        uint8_t* prow = smem + Ly::OFF_P + w * Ly::P_BYTES + r * 128;
+        uint32_t pk[TN / 2];
 #pragma unroll
-        for (int pc = 0; pc < 8; ++pc) {
-          uint4 v;
-          v.x = pack_bf16x2(x[8 * pc + 0], x[8 * pc + 1]);
-          v.y = pack_bf16x2(x[8 * pc + 2], x[8 * pc + 3]);
-          v.z = pack_bf16x2(x[8 * pc + 4], x[8 * pc + 5]);
-          v.w = pack_bf16x2(x[8 * pc + 6], x[8 * pc + 7]);
-          *reinterpret_cast<uint4*>(prow + ((pc ^ (r & 7)) * 16)) = v;
-        }
-        fence_proxy_async_smem();
+        for (int c = 0; c < TN / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+        tmem_st32(t_s, pk);  // P over the first TN / 2 columns of its S buffer
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(w));
+        if (lane == 0) mbar_arrive(p_full(2 * gb + half));
+        prev_gi = gi;
       }
 
       if (last) {
@@ -538,6 +878,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         ++pieces;
       }
+      if (group_last(cur, j, n)) ++gi;
       cursor_next(cur, p);
     }
   }
@@ -550,100 +891,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-}
 
-// Merge the pieces of each (sequence, KV head, head chunk) segment by
-// log-sum-exp.  One warp per query row; lane owns D/32 consecutive columns.
-// The pieces' (m, l) pairs are read lane-parallel and their O rows are
-// fetched with independent loads so the merge is bandwidth-, not
-// latency-bound.
-template <int D>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const Params p, int grid_ctas,
-                                                           __nv_bfloat16* __restrict__ out) {
-  constexpr int PER = D / 32;
-  const int s = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r = blockIdx.y * 4 + warp;
-  const int nseg = p.Hkv * p.nhc;
-  const int b = s / nseg, seg = s % nseg;
-  const int g = seg / p.nhc, hc = seg % p.nhc;
-  const int i = r / p.Gc, hh = r % p.Gc;
-  if (i >= p.K || hc * p.Gc + hh >= p.G) return;
-
-  long long T = 0, Ts = 0;
-  int nt_b = 1;
-  for (int bb = 0; bb < p.B; ++bb) {
-    const int nt = n_tiles(clamp_len(__ldg(p.ctx_lens + bb), p), p);
-    if (bb == b) {
-      Ts = T + static_cast<long long>(seg) * nt;
-      nt_b = nt;
-    }
-    T += static_cast<long long>(nseg) * nt;
+  // Every CTA's partials are written: meet at the grid barrier, then merge an
+  // equal share of the output rows.  Thread 0 first records which CTAs hold
+  // pieces of the segments of this CTA's rows (into the now idle K ring).
+  const int RV = p.Gc * p.K;
+  const long long R = static_cast<long long>(p.B) * nseg * RV;
+  const long long r0 = mul_div(blockIdx.x, R, gridDim.x);
+  const long long r1 = mul_div(blockIdx.x + 1, R, gridDim.x);
+  SegPieces* segs = reinterpret_cast<SegPieces*>(smem + Ly::OFF_K);
+  const long long s_first = mul_div(r0, 1, RV);
+  const long long s_last = r1 > r0 ? mul_div(r1 - 1, 1, RV) : s_first - 1;
+  const int n_segs = static_cast<int>(s_last - s_first + 1 < MERGE_SEGS ? s_last - s_first + 1
+                                                                        : MERGE_SEGS);
+  if (threadIdx.x == 0) {
+    const unsigned long long target = grid_arrive(p.gbar, gridDim.x);
+    for (int k = 0; k < n_segs; ++k) segs[k] = segment_pieces(p, gridDim.x, s_first + k);
+    grid_wait(p.gbar, target, p.dev_status);
   }
-  const long long P = grid_ctas;
-  const long long c0 = cta_of(Ts, T, P), c1 = cta_of(Ts + nt_b - 1, T, P);
-
-  float M = -INFINITY;
-  for (long long base = c0; base <= c1; base += 32) {
-    const long long c = base + lane;
-    if (c <= c1 && cta_start(c, T, P) != cta_start(c + 1, T, P))
-      M = fmaxf(M, __ldcg(&p.part_ml[(s + c) * ROWS + r]).x);
-  }
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, m));
-
-  float acc[PER];
-#pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  float Lp = 0.f;
-  for (long long base = c0; base <= c1; base += 32) {
-    const long long c = base + lane;
-    float wgt = 0.f;
-    if (c <= c1 && cta_start(c, T, P) != cta_start(c + 1, T, P)) {
-      const float2 ml = __ldcg(&p.part_ml[(s + c) * ROWS + r]);
-      wgt = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - M);
-      Lp += wgt * ml.y;
-    }
-    const int cnt = static_cast<int>(c1 - base + 1 < 32 ? c1 - base + 1 : 32);
-    for (int k0 = 0; k0 < cnt; k0 += 8) {
-      // eight independent loads in flight, then the weighted sums
-      float wk[8];
-      float v[8][PER];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        wk[k] = __shfl_sync(0xFFFFFFFFu, wgt, (k0 + k) & 31);
-        const bool live = (k0 + k < cnt) && wk[k] != 0.f;
-        const float* src = p.part_o + ((s + base + k0 + k) * ROWS + r) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 t = live ? __ldcg(reinterpret_cast<const float4*>(src))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[k][0] = t.x;
-          v[k][1] = t.y;
-          v[k][2] = t.z;
-          v[k][3] = t.w;
-        } else {
-          const float2 t = live ? __ldcg(reinterpret_cast<const float2*>(src))
-                                : make_float2(0.f, 0.f);
-          v[k][0] = t.x;
-          v[k][1] = t.y;
-        }
-        if (!live) wk[k] = 0.f;
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-#pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += wk[k] * v[k][e];
-    }
-  }
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) Lp += __shfl_xor_sync(0xFFFFFFFFu, Lp, m);
-  const float inv = Lp > 0.f ? 1.f / Lp : 0.f;
-  const int h = g * p.G + hc * p.Gc + hh;
-  __nv_bfloat16* dst = out + ((static_cast<long long>(b) * p.K + i) * p.Hq + h) * D + lane * PER;
-#pragma unroll
-  for (int k = 0; k < PER; k += 2)
-    *reinterpret_cast<__nv_bfloat162*>(dst + k) = __floats2bfloat162_rn(acc[k] * inv,
-                                                                        acc[k + 1] * inv);
+  __syncthreads();
+  merge_rows<D>(p, gridDim.x, r0, r1, warp, THREADS / 32, lane, segs, s_first, n_segs);
 }
 
 struct Shape {
@@ -668,17 +935,21 @@ int check_shape(int B, int Hq, int Hkv, int d, int K, Shape* sh) {
   return ORTHRUS_OK;
 }
 
+// Workspace: [0, 256) grid-barrier words (must be zero before the first use;
+// every call leaves them zero), then the partial O and (m, l) of every piece.
+constexpr size_t WS_HEADER = 256;
+
 size_t workspace_bytes(const Shape& sh, int sms) {
   const size_t slots = static_cast<size_t>(sh.S) + static_cast<size_t>(sms);
   const size_t o_bytes = slots * ROWS * sh.d * sizeof(float);
   const size_t ml_bytes = slots * ROWS * sizeof(float2);
-  return o_bytes + ml_bytes + 256;
+  return WS_HEADER + o_bytes + ml_bytes;
 }
 
 template <int D>
 int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int mask_mode,
            void* out, void* ws, int sms, int32_t* dev_status, cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq;
   {
     const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(sh.Hq),
                               static_cast<uint64_t>(sh.B) * sh.K};
@@ -688,22 +959,27 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
     const int rc = encode_tmap_bf16(&tq, q, 3, dims, strides, box);
     if (rc != ORTHRUS_OK) return rc;
   }
+  CUtensorMap tk2, tk1, tv2, tv1;
   {
     const uint64_t dims[2] = {static_cast<uint64_t>(D),
                               static_cast<uint64_t>(sh.B) * sh.Hkv * cache->cap};
     const uint64_t strides[1] = {static_cast<uint64_t>(D) * 2};
-    const uint32_t box[2] = {64u, static_cast<uint32_t>(TN)};
-    int rc = encode_tmap_bf16(&tk, cache->k, 2, dims, strides, box);
-    if (rc != ORTHRUS_OK) return rc;
-    rc = encode_tmap_bf16(&tv, cache->v, 2, dims, strides, box);
+    const uint32_t box2[2] = {64u, static_cast<uint32_t>(2 * TN)};
+    const uint32_t box1[2] = {64u, static_cast<uint32_t>(TN)};
+    int rc = encode_tmap_bf16(&tk2, cache->k, 2, dims, strides, box2);
+    if (rc == ORTHRUS_OK) rc = encode_tmap_bf16(&tk1, cache->k, 2, dims, strides, box1);
+    if (rc == ORTHRUS_OK) rc = encode_tmap_bf16(&tv2, cache->v, 2, dims, strides, box2);
+    if (rc == ORTHRUS_OK) rc = encode_tmap_bf16(&tv1, cache->v, 2, dims, strides, box1);
     if (rc != ORTHRUS_OK) return rc;
   }
   Params p;
   p.ctx_lens = cache->ctx_lens;
   const size_t slots = static_cast<size_t>(sh.S) + static_cast<size_t>(sms);
   uint8_t* w = static_cast<uint8_t*>(ws);
-  p.part_o = reinterpret_cast<float*>(w);
-  p.part_ml = reinterpret_cast<float2*>(w + slots * ROWS * D * sizeof(float));
+  p.gbar = reinterpret_cast<unsigned long long*>(w);
+  p.part_o = reinterpret_cast<float*>(w + WS_HEADER);
+  p.part_ml = reinterpret_cast<float2*>(w + WS_HEADER + slots * ROWS * D * sizeof(float));
+  p.out = static_cast<__nv_bfloat16*>(out);
   p.dev_status = dev_status;
   p.B = sh.B;
   p.K = sh.K;
@@ -718,11 +994,20 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
 
   auto* kfn = attn_splitkv_kernel<D>;
   if (!opt_in_smem(reinterpret_cast<const void*>(kfn), Layout<D>::ALLOC)) return ORTHRUS_ECUDA;
-  kfn<<<sms, THREADS, Layout<D>::ALLOC, stream>>>(tq, tk, tv, p);
-  if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
-  const dim3 cgrid(sh.S, (sh.Gc * sh.K + 3) / 4);
-  attn_combine_kernel<D><<<cgrid, 128, 0, stream>>>(p, sms, static_cast<__nv_bfloat16*>(out));
-  if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
+  // Cooperative launch: the grid barrier before the merge needs every CTA
+  // resident at once (one CTA per SM).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Layout<D>::ALLOC;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p) != cudaSuccess)
+    return ORTHRUS_ECUDA;
   return ORTHRUS_OK;
 }
 

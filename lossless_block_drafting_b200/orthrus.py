@@ -125,6 +125,12 @@ def block_attn_workspace_size(B: int, Hq: int, Hkv: int, d: int, K: int) -> int:
     return int(n.value)
 
 
+def new_block_attn_workspace(B: int, Hq: int, Hkv: int, d: int, K: int, device=None):
+    """A zero-filled workspace for block_attn (its barrier words must start at 0)."""
+    return torch.zeros(block_attn_workspace_size(B, Hq, Hkv, d, K), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
 def block_attn(q, k_cache, v_cache, ctx_lens, mask_mode: int, out=None, workspace=None,
                dev_status=None, stream=None, cache_view: KVCacheView | None = None):
     """Block-query attention: q bf16 [B,K,Hq,d] over the cache -> bf16 [B,K,Hq,d]."""
@@ -136,8 +142,7 @@ def block_attn(q, k_cache, v_cache, ctx_lens, mask_mode: int, out=None, workspac
     else:
         _need(out, torch.bfloat16, "out", 4)
     if workspace is None:
-        workspace = torch.empty(block_attn_workspace_size(B, Hq, view.Hkv, d, K),
-                                dtype=torch.uint8, device=q.device)
+        workspace = new_block_attn_workspace(B, Hq, view.Hkv, d, K, q.device)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_block_attn(_ptr(q), ctypes.byref(view), Hq, K, int(mask_mode), _ptr(out),

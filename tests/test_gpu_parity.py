@@ -64,6 +64,8 @@ ATTN_CASES = [
     (2, 32, 32, 8, 128, [1000, 257], 1400),         # Qwen3-8B heads, ragged
     (1, 16, 16, 2, 64, [300], None),               # G*K = 128 exactly
     (2, 32, 16, 2, 128, [100, 70], None),          # G*K = 256 -> two head chunks
+    (1, 8, 4, 1, 64, [50], None),                  # one short segment: most CTAs idle
+    (20, 4, 16, 8, 64, list(range(60, 1260, 60)), None),  # 160 segments > 148 CTAs
 ]
 
 
@@ -130,12 +132,14 @@ def test_block_attn_repeat_calls_same_workspace_are_deterministic():
     case = synth.attn_case(2, 32, 32, 8, 128, [3000, 5000], seed=8)
     q, kc, vc = case.q.cuda(), case.k_cache.cuda(), case.v_cache.cuda()
     cl = torch.from_numpy(case.ctx_lens).cuda()
-    ws = torch.empty(ob.block_attn_workspace_size(2, 32, 8, 128, 32), dtype=torch.uint8,
-                     device="cuda")
+    ws = torch.zeros(ob.block_attn_workspace_size(2, 32, 8, 128, 32), dtype=torch.uint8, device="cuda")
     a = ob.block_attn(q, kc, vc, cl, ob.MASK_AR, workspace=ws).clone()
     b = ob.block_attn(q, kc, vc, cl, ob.MASK_AR, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+    # the grid-barrier ticket counter advanced by exactly one grid per call
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert int(ws[:8].view(torch.int64).item()) == 2 * sms
 
 
 def _check_argmax(got, ref_am, gap):
