@@ -44,7 +44,7 @@ def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ctx", type=int, default=40960)
@@ -70,6 +70,62 @@ def dist_env():
     return rank, world, local
 
 
+ATTN_SOURCES = ("lossless_block_drafting_b200/csrc/block_attn.cu",
+                "lossless_block_drafting_b200/csrc/common.cuh",
+                "lossless_block_drafting_b200/csrc/ptx.cuh")
+
+
+def attn_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(wl):
+    """DRAM bytes (read + write) per attention launch from the committed ncu
+    capture, scaled to this workload's KV bytes; None once the kernel's sources
+    differ from the ones the counters were taken on, or for another workload."""
+    path = os.path.join(ROOT, "profiles", "block_attn_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != attn_source_hash():
+        return None
+    if (rec.get("ctx"), rec.get("block_K"), rec.get("batch")) != (wl.L0, wl.K, wl.B):
+        return None
+    return int(rec["dram_bytes_read"] + rec["dram_bytes_write"])
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Largest value over all ranks (identity without a process group).
+
+    Timings are reduced this way so the slowest replica sets the step time.
+    """
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sync_ranks():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.barrier()
+
+
+def weak_scaling_value(tokens_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job verified tokens/s: every replica verifies tokens_per_rank per step."""
+    return world * tokens_per_rank / (max_ms * 1e-3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -84,7 +140,7 @@ def peaks():
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -98,7 +154,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -108,9 +164,13 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
-    def stop(self):
+    def mark(self):
+        """Host time stamp; samples between two marks form the timed window."""
+        return time.time()
+
+    def stop(self, t0=None, t1=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -122,16 +182,20 @@ class ClockSampler:
             self._t.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        window = [(ts, ln) for ts, ln in self.lines
+                  if (t0 is None or ts >= t0) and (t1 is None or ts <= t1 + 0.05)]
+        if not window:  # window shorter than the sampling period: nearest samples
+            window = self.lines[-3:]
+        for _, ln in window:
             parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
+                sm.append(float(parts[2]))
+                smax.append(float(parts[3]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            for n, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
@@ -185,11 +249,11 @@ class Workload:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.views = [ob.kv_cache_view(self.k[i], self.v[i], self.ctx_lens) for i in range(layers)]
 
-    # kernels launched per step (main + combine per attention call; main +
-    # reduce per LM head; one verify+commit)
+    # kernels launched per step (one per attention call; main + reduce per LM
+    # head; one verify+commit)
     @property
     def launches_per_step(self):
-        return 2 * self.layers * 2 + 2 * 2 + 1
+        return 2 * self.layers + 2 * 2 + 1
 
     def attn_bytes(self):
         """Algorithmic bytes of one attention call at the starting context."""
@@ -287,24 +351,20 @@ def run_ours(args):
     sampler = ClockSampler(dev.index)
     if rank == 0:
         sampler.start()
-    if world > 1:
-        dist.barrier()
+    sync_ranks()
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    t_win0 = time.time()
     with torch.cuda.stream(stream):
         start.record(stream)
         g_timed.replay()
         end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if rank == 0 else None
-    ms_total = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    t_win1 = time.time()
+    sync_ranks()
+    clocks = sampler.stop(t_win0, t_win1) if rank == 0 else None
+    ms_total = max_over_ranks(start.elapsed_time(end), dev)
     ms_step = ms_total / K_steps
 
     # per-phase times from the event nodes of every timed step
@@ -321,7 +381,7 @@ def run_ours(args):
     status = int(wl.status.item())
 
     tokens = wl.B * wl.K
-    value = world * tokens / (ms_step * 1e-3)
+    value = weak_scaling_value(tokens, world, ms_step)
     attn_gbs = wl.attn_bytes() / (attn_us * 1e-6) / 1e9
     lm_gbs = wl.lm_bytes() / (lm_us * 1e-6) / 1e9
     lm_tflops = 2.0 * wl.B * wl.K * wl.H * wl.V / (lm_us * 1e-6) / 1e12
@@ -362,7 +422,7 @@ def run_ours(args):
         "breakdown_ms_per_step": {k: round(v, 4) for k, v in ph.items()},
         "verify_pass_only": {
             "ms": round(verify_pass_ms, 4),
-            "tokens_per_s": round(world * tokens / (verify_pass_ms * 1e-3), 2),
+            "tokens_per_s": round(weak_scaling_value(tokens, world, verify_pass_ms), 2),
         },
         "attn": {"us_per_call": round(attn_us, 2), "GB_per_s": round(attn_gbs, 1),
                  "frac_of_hbm_peak": round(attn_gbs / hbm_peak, 4)},
@@ -371,7 +431,8 @@ def run_ours(args):
                    "frac_of_hbm_peak": round(lm_gbs / hbm_peak, 4),
                    "frac_of_bf16_peak": round(lm_tflops / tc_sus, 4)},
         "roofline": {
-            "kernel": "orthrus_block_attn (split-KV main + LSE combine), AR and DIFF masks",
+            "kernel": "orthrus_block_attn (cooperative split-KV kernel with in-kernel LSE merge), "
+                      "AR and DIFF masks",
             "bound": "hbm",
             "achieved": round(attn_gbs, 1),
             "peak": hbm_peak,
@@ -379,7 +440,7 @@ def run_ours(args):
                            if peak_kind == "measured" else "fallback 6650 GB/s",
             "unit": "GB/s",
             "frac": round(attn_gbs / hbm_peak, 4),
-            "traffic": None,
+            "traffic": measured_traffic(wl),
             "algorithmic_bytes_per_launch": wl.attn_bytes(),
         },
         "gpu_launches": wl.launches_per_step * K_steps,
@@ -393,7 +454,7 @@ def run_ours(args):
     if args.sweep and rank == 0:
         result["sweep"] = run_sweep(dev, stream)
     if world > 1:
-        dist.barrier()
+        sync_ranks()
         dist.destroy_process_group()
     return result if rank == 0 else None
 
@@ -426,9 +487,7 @@ def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):
     for _ in range(W_steps):
         one()
     torch.cuda.synchronize()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    sync_ranks()
     t0 = time.perf_counter()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -437,14 +496,9 @@ def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):
         one()
     end.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / K_steps
+    ms = max_over_ranks(start.elapsed_time(end) / K_steps, dev)
     wall_ms = (time.perf_counter() - t0) * 1e3 / K_steps
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return {"value": round(world * wl.B * wl.K / (ms * 1e-3), 2), "unit": UNIT,
+    return {"value": round(weak_scaling_value(wl.B * wl.K, world, ms), 2), "unit": UNIT,
             "ms_per_step": round(ms, 4), "host_wall_ms_per_step": round(wall_ms, 4),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
