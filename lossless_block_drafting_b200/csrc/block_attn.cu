@@ -263,12 +263,11 @@ __device__ void grid_wait(unsigned long long* gbar, unsigned long long target,
                           int32_t* status) {
   volatile unsigned long long* v = gbar;
   const uint64_t t0 = globaltimer_ns();
-  while (*v < target) {
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+  for (uint32_t polls = 0; *v < target; ++polls) {
+    if ((polls & 255u) == 255u && globaltimer_ns() - t0 > kWaitTimeoutNs) {
       report(status, ORTHRUS_ETIMEOUT);
       break;
     }
-    __nanosleep(32);
   }
   __threadfence();
 }
@@ -329,7 +328,7 @@ __device__ SegPieces segment_pieces(const Params& p, int P, long long s) {
 constexpr int MERGE_SEGS = 64;  // segment records precomputed per CTA
 
 // Merge the pieces of output rows [r0, r1) (flat over segments x rows of a
-// segment) by log-sum-exp; one warp per row, lane owns D/32 columns, twelve
+// segment) by log-sum-exp; one warp per row, lane owns D/32 columns, up to 12
 // pieces' loads in flight per round.  Segment records for the CTA's rows are
 // in `segs` (first segment s_first, n_segs of them); rows beyond them fall
 // back to computing the record in lane 0.
@@ -502,6 +501,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
     tmem_relinquish();
+  }
+  {
+    // Query rows past the Gc*K real ones are never loaded: zero them once so
+    // their scores are plain zeros (whole 128-byte rows, swizzle-invariant).
+    const int first_pad = p.Gc * p.K;
+    const int pieces16 = (ROWS - first_pad) * 8 * Ly::CHUNKS;
+    for (int q = threadIdx.x; q < pieces16; q += THREADS) {
+      const int ch = q / ((ROWS - first_pad) * 8), rem = q % ((ROWS - first_pad) * 8);
+      *reinterpret_cast<uint4*>(smem + Ly::OFF_Q + ch * Ly::Q_CHUNK +
+                                (first_pad + rem / 8) * 128 + (rem % 8) * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -697,11 +709,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t t_o = lane_base + TMEM_O + w * 128;
     const int rows_valid = p.Gc * p.K;
     const int i_row = r / p.Gc;
+    const bool idle_warp = (warp & 3) * 32 >= rows_valid;
     const float sl2 = p.sl2;
     Cursor cur;
     cur = start;
     int pieces = 0, jp = 0, gi = 0, prev_gi = 0;
     float m_used = -INFINITY, l_sum = 0.f;
+    // A tile that runs past the valid keys: the warpgroup's 128 threads zero
+    // those V rows together, so that stale or NaN cache contents cannot reach
+    // O through 0 * NaN.  Returns false if the V stage never arrived.
+    auto zero_v_tail = [&](int tile0, int kv_end, bool first_half) -> bool {
+      const int stage = gi % NV;
+      if (!mbar_wait_warp(full_v(stage), (gi / NV) & 1, abort_flag, p.dev_status)) return false;
+      const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
+      const int per_chunk = (TN - nv) * 8;
+      uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES + (first_half ? 0 : Ly::HALF);
+      for (int q = r; q < per_chunk * Ly::CHUNKS; q += ROWS) {
+        const int ch = q / per_chunk, rem = q % per_chunk;
+        *reinterpret_cast<uint4*>(vt + ch * Ly::KV_CHUNK + (nv + rem / 8) * 128 +
+                                  (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      return true;
+    };
     for (int j = 0; j < n; ++j) {
       const bool first = (j == 0) || cur.t == 0;
       const bool last = (j == n - 1) || cur.t == cur.nt - 1;
@@ -710,7 +740,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = -INFINITY;
         l_sum = 0.f;
       }
-      if ((j & 1) == w) {
+      if ((j & 1) == w && idle_warp) {
+        // All 32 rows of this warp are padding: no softmax, but it still
+        // waits for S (which keeps it within one phase of the P barriers),
+        // takes its share of a tail tile's V zeroing, and arrives so the P*V
+        // issuer's count is complete.  The P rows it leaves unwritten feed
+        // only padding rows of O, which are never read.
+        WARP_WAIT_OR(s_full(gi & 1), (gi >> 1) & 1, break);
+        const int tile0 = cur.t * TN;
+        const int kv_end = cur.L + p.K;
+        if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, group_first(cur, j))) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(2 * (gi & 1) + (group_first(cur, j) ? 0 : 1)));
+        prev_gi = gi;
+      } else if ((j & 1) == w) {
         const bool fresh = (j - jp) < 2;
         const int gb = gi & 1;
         const int half = group_first(cur, j) ? 0 : 1;
@@ -773,9 +816,32 @@ __global__ void __launch_bounds__(THREADS, 1)
           m_used = reduce_max();
           exps(m_used, false);
         } else {
-          exps(m_used, true);
-          const float mx = reduce_max();
-          if (__any_sync(0xFFFFFFFFu, mx > m_used + 8.f)) {
+          // Every p is positive, so a tile row sum of at most 2^8 proves no
+          // element exceeded the reference by more than 2^8: the sums the row
+          // needs anyway decide whether the (rare) rescale path runs, and only
+          // then is the tile max taken.
+          exps(m_used, false);
+          const float2 ts2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
+          if (__any_sync(0xFFFFFFFFu, !(ts2.x + ts2.y <= 256.f))) {
+            // S is still in its TMEM buffer: reload it (re-masked), take the
+            // tile max, rescale O_w and l, and redo the tile.
+            tmem_ld64(t_s, sr);
+            tmem_wait_ld();
+            if (tile0 + TN > cur.L + 1) {
+              const int lim = (r >= rows_valid) ? 0
+                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+#pragma unroll
+              for (int c = 0; c < TN; ++c)
+                if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int c = 0; c < TN; c += 8) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
+                               __uint_as_float(sr[c + 2 * q + 1]));
+            }
+            const float mx = reduce_max();
             const float m_new = fmaxf(m_used, mx);
             const float f = (m_new == -INFINITY) ? 1.f
                             : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
@@ -795,38 +861,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_wait_st();
             l_sum *= f;
             m_used = m_new;
-            // S is still in its TMEM buffer: reload it (re-masked) and redo
-            tmem_ld64(t_s, sr);
-            tmem_wait_ld();
-            if (tile0 + TN > cur.L + 1) {
-              const int lim = (r >= rows_valid) ? 0
-                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
-#pragma unroll
-              for (int c = 0; c < TN; ++c)
-                if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-            }
             exps(m_used, false);
           }
         }
         const float2 t2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
         l_sum += t2.x + t2.y;
 
-        if (tile0 + TN > kv_end) {
-          // The tile runs past the valid keys: zero those V rows so that stale
-          // or NaN cache contents cannot reach O through 0 * NaN.
-          const int stage = gi % NV;
-          WARP_WAIT_OR(full_v(stage), (gi / NV) & 1, break);
-          const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
-          const int per_chunk = (TN - nv) * 8;
-          uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES +
-                        (group_first(cur, j) ? 0 : Ly::HALF);
-          for (int q = r; q < per_chunk * Ly::CHUNKS; q += ROWS) {
-            const int ch = q / per_chunk, rem = q % per_chunk;
-            *reinterpret_cast<uint4*>(vt + ch * Ly::KV_CHUNK + (nv + rem / 8) * 128 +
-                                      (rem % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-        }
+        if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, group_first(cur, j))) break;
         uint32_t pk[TN / 2];
 #pragma unroll
         for (int c = 0; c < TN / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
@@ -851,27 +892,29 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
           const long long slot = static_cast<long long>(cur.b) * nseg + cur.seg + blockIdx.x;
           float* dst = p.part_o + (slot * ROWS + r) * D;
+          if (!idle_warp) {  // rows of all-padding warps are never merged
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o0[32], o1r[32];
-            tmem_ld32(t_o + c0, o0);
-            tmem_ld32(t_o + 128 + c0, o1r);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o0[32], o1r[32];
+              tmem_ld32(t_o + c0, o0);
+              tmem_ld32(t_o + 128 + c0, o1r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 32; k += 4) {
-              float4 v;
-              v.x = (a0 != 0.f ? a0 * __uint_as_float(o0[k]) : 0.f) +
-                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k]) : 0.f);
-              v.y = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 1]) : 0.f) +
-                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 1]) : 0.f);
-              v.z = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 2]) : 0.f) +
-                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
-              v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
-                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
-              *reinterpret_cast<float4*>(dst + c0 + k) = v;
+              for (int k = 0; k < 32; k += 4) {
+                float4 v;
+                v.x = (a0 != 0.f ? a0 * __uint_as_float(o0[k]) : 0.f) +
+                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k]) : 0.f);
+                v.y = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 1]) : 0.f) +
+                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 1]) : 0.f);
+                v.z = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 2]) : 0.f) +
+                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
+                v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
+                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
+                *reinterpret_cast<float4*>(dst + c0 + k) = v;
+              }
             }
+            p.part_ml[slot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
           }
-          p.part_ml[slot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(o_free);
