@@ -115,19 +115,22 @@ int orthrus_block_attn_workspace_size(int B, int Hq, int Hkv, int d, int K, size
  *   Hq, K      query heads (multiple of cache->Hkv), block size 1..32
  *   mask_mode  orthrus_mask_mode
  *   out        bf16 [B, K, Hq, d] device
- *   workspace  device, >= orthrus_block_attn_workspace_size(...) bytes.  Its
- *              first 256 bytes (a grid-barrier counter) must be zero before the
- *              first call; afterwards each call advances the counter by the
- *              grid size, which keeps it consistent for the next call (zero it
- *              again after an ORTHRUS_ETIMEOUT, and before using the workspace
- *              on a device with a different SM count).  The rest may hold
- *              anything.  Calls that share a workspace must be stream-ordered.
+ *   workspace  device, >= orthrus_block_attn_workspace_size(...) bytes, zero
+ *              filled before the first call.  Its head holds a grid-barrier
+ *              counter and one completion counter per (sequence, KV head, head
+ *              chunk) segment; each call advances every counter it uses by a
+ *              fixed amount, which keeps them consistent for the next call, so
+ *              a workspace is zeroed once, not per call (zero it again after an
+ *              ORTHRUS_ETIMEOUT, and before using it on a device with a
+ *              different SM count).  The rest holds per-call partial results.
+ *              Calls that share a workspace must be stream-ordered.
  *   dev_status int32 device or NULL (see conventions; ORTHRUS_ECAPACITY when
  *              L_b + K > cap, in which case L_b is clamped to cap - K)
  * Supported: d in {64, 128}; 1 <= K <= 32; Hq / Hkv <= 128.
  * Runs as one cooperative, persistent split-KV kernel (one CTA per SM, tcgen05
  * MMAs with TMEM accumulators, TMA-staged K/V tiles) whose CTAs merge their
- * partial results by log-sum-exp after a grid barrier.
+ * partial results by log-sum-exp: per segment, behind that segment's counter,
+ * when every segment gets its own CTAs; after a grid barrier otherwise.
  */
 int orthrus_block_attn(const void *q, const orthrus_kv_cache *cache, int Hq, int K,
                        int mask_mode, void *out, void *workspace, size_t ws_bytes,

@@ -74,8 +74,8 @@ struct Layout {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;  // [ROWS] float2 handed WG1 -> WG0
-  static constexpr int OFF_SCHED = OFF_ML + ROWS * 8;  // 6 x int64 CTA schedule
-  static constexpr int OFF_BAR = OFF_SCHED + 64;
+  static constexpr int OFF_SCHED = OFF_ML + ROWS * 8;  // 9 x int64 CTA schedule
+  static constexpr int OFF_BAR = OFF_SCHED + 128;
   static constexpr int NBAR = 2 * NK + 2 * NV + 13;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
@@ -87,6 +87,7 @@ struct Params {
   float* part_o;      // [slots][ROWS][D] unnormalised O of each piece
   float2* part_ml;    // [slots][ROWS] (m in log2 units, l)
   unsigned long long* gbar;  // grid-barrier arrival ticket counter (starts at 0)
+  unsigned long long* seg_cnt;  // [S] per-segment completion counters (start at 0)
   __nv_bfloat16* out; // [B, K, Hq, D]
   int32_t* dev_status;
   int B, K, Hq, Hkv, G, Gc, nhc, cap, mask_mode;
@@ -216,20 +217,28 @@ __device__ __forceinline__ long long cta_of(long long x, long long T, long long 
   return mul_div((x + 1) * P - 1, 1, T);
 }
 
-// Flat tile range [x0, x1) of CTA c.
+// Flat tile range [x0, x1) of CTA c.  Under the per-segment partition *own
+// receives the CTA's segment (flat index, its CTAs and tiles).
+struct OwnSeg {
+  long long s;
+  int c0, cn, ns;
+};
+
 __device__ void cta_range(const Params& p, long long T, int P, int c, long long* x0,
-                          long long* x1) {
+                          long long* x1, OwnSeg* own) {
   if (!segment_partition(p, P)) {
     *x0 = cta_start(c, T, P);
     *x1 = cta_start(c + 1, T, P);
     return;
   }
   *x0 = *x1 = T;
+  const int nseg = p.Hkv * p.nhc;
   walk_segments(p, T, P, [&](const SegWalk& w) {
     if (c < w.c0 || c >= w.c0 + w.cn) return false;
     const long long k = c - w.c0;
     *x0 = w.Ts + mul_div(k, w.ns, w.cn);
     *x1 = w.Ts + mul_div(k + 1, w.ns, w.cn);
+    *own = OwnSeg{static_cast<long long>(w.b) * nseg + w.seg, w.c0, w.cn, w.ns};
     return true;
   });
 }
@@ -421,6 +430,142 @@ __device__ void merge_rows(const Params& p, int P, long long r0, long long r1, i
   }
 }
 
+// Per-segment partition: CTA k of the cn CTAs of segment s merges rows
+// [row0, row1) of that segment, RC rows per round.  One thread bulk-copies the
+// rows' fp32 partial O of up to NPB pieces into shared memory (one contiguous
+// copy per piece, all in flight at once) while every thread loads one (m, l);
+// one warp per row turns the m's into weights against the running row max,
+// then thread (row, float4 column) accumulates the weighted partials and
+// finally writes O / l as bf16.  `buf` is the idle K/V ring (1024-aligned).
+template <int D>
+__device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int row1, int warp,
+                              int lane, uint8_t* buf, volatile int* abort_flag) {
+  constexpr int RC = 8;                                  // rows per round
+  constexpr int Q4 = D / 4;                              // float4 columns of a row
+  constexpr int PIECE = RC * D * 4;                      // bytes of one piece's rows
+  constexpr int HEAD = 8192;                             // barrier, weights, row state
+  constexpr int AVAIL = (Layout<D>::NK + Layout<D>::NV) * Layout<D>::KV_BYTES - HEAD;
+  constexpr int NPB = AVAIL / PIECE < THREADS / RC ? AVAIL / PIECE : THREADS / RC;
+  static_assert(NPB >= 1 && NPB <= 64, "merge batch: 1..64 pieces (two per lane of warp 0)");
+  const uint32_t bar = smem_u32(buf);
+  float2* ml_s = reinterpret_cast<float2*>(buf + 64);                        // [NPB][RC]
+  float* w_s = reinterpret_cast<float*>(buf + 64 + NPB * RC * 8);             // [NPB][RC]
+  float* row_s = reinterpret_cast<float*>(buf + 64 + NPB * RC * 12);          // M, L, scale
+  const float4* o_s = reinterpret_cast<const float4*>(buf + HEAD);            // [NPB][RC][Q4]
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool dense = own.cn <= own.ns;  // every CTA of the segment wrote a piece
+  auto live = [&](int j) {
+    return dense || mul_div(j, own.ns, own.cn) != mul_div(j + 1, own.ns, own.cn);
+  };
+  const int nseg = p.Hkv * p.nhc;
+  const int b = static_cast<int>(own.s / nseg), seg = static_cast<int>(own.s % nseg);
+  const int g = seg / p.nhc, hc = seg % p.nhc;
+  uint32_t phase = 0;
+  for (int rb = row0; rb < row1; rb += RC) {
+    const int nr = row1 - rb < RC ? row1 - rb : RC;
+    if (threadIdx.x < RC) {
+      row_s[threadIdx.x] = -INFINITY;       // running max
+      row_s[RC + threadIdx.x] = 0.f;        // running normaliser
+    }
+    const int tr = threadIdx.x / Q4, tq = threadIdx.x % Q4;  // this thread's (row, float4)
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < own.cn; j0 += NPB) {
+      const int nb = own.cn - j0 < NPB ? own.cn - j0 : NPB;
+      if (warp == 0) {
+        // Lane l copies pieces l and l + 32 of the batch (issue is parallel:
+        // one bulk copy costs ~150 cycles of issue in a single thread).
+        const bool on0 = lane < nb && live(j0 + lane);
+        const bool on1 = lane + 32 < nb && live(j0 + lane + 32);
+        const uint32_t n_on = __popc(__ballot_sync(0xFFFFFFFFu, on0)) +
+                              __popc(__ballot_sync(0xFFFFFFFFu, on1));
+        if (lane == 0) mbar_arrive_expect_tx(bar, n_on * nr * D * 4);
+        __syncwarp();
+        if (on0 || on1) fence_proxy_async_global();  // partials were written by generic stores
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (!(u == 0 ? on0 : on1)) continue;
+          const int jj = lane + 32 * u;
+          const long long slot = own.s + own.c0 + j0 + jj;
+          bulk_load(smem_u32(buf + HEAD + jj * PIECE), p.part_o + (slot * ROWS + rb) * D,
+                    nr * D * 4, bar);
+        }
+      }
+      if (threadIdx.x < nb * RC) {
+        const int jj = threadIdx.x / RC, r = threadIdx.x % RC;
+        const long long slot = own.s + own.c0 + j0 + jj;
+        ml_s[threadIdx.x] = (r < nr && live(j0 + jj)) ? __ldcg(p.part_ml + slot * ROWS + rb + r)
+                                                      : make_float2(-INFINITY, 0.f);
+      }
+      __syncthreads();
+      if (warp < nr) {
+        // Row `warp`: batch max, weights, running (M, L) and the rescale of acc.
+        const int r = warp;
+        float mb = -INFINITY;
+        for (int jj = lane; jj < nb; jj += 32) mb = fmaxf(mb, ml_s[jj * RC + r].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        const float m_old = row_s[r];
+        const float m_new = fmaxf(m_old, mb);
+        float lb = 0.f;
+        for (int jj = lane; jj < nb; jj += 32) {
+          const float2 ml = ml_s[jj * RC + r];
+          const float wj = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - m_new);
+          w_s[jj * RC + r] = wj;
+          lb += wj * ml.y;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) lb += __shfl_xor_sync(0xFFFFFFFFu, lb, o);
+        if (lane == 0) {
+          const float sc = m_old == -INFINITY ? 0.f : fast_exp2(m_old - m_new);
+          row_s[r] = m_new;
+          row_s[RC + r] = row_s[RC + r] * sc + lb;
+          row_s[2 * RC + r] = sc;
+        }
+      }
+      mbar_wait_bounded(bar, phase, abort_flag, p.dev_status);  // gives up: status set
+      phase ^= 1u;
+      __syncthreads();
+      if (tr < nr) {
+        const float sc = row_s[2 * RC + tr];
+        acc.x *= sc;
+        acc.y *= sc;
+        acc.z *= sc;
+        acc.w *= sc;
+        for (int jj = 0; jj < nb; ++jj) {
+          const float wj = w_s[jj * RC + tr];
+          if (wj == 0.f) continue;  // dead piece or no mass: its rows may be stale
+          const float4 x = o_s[(jj * RC + tr) * Q4 + tq];
+          acc.x += wj * x.x;
+          acc.y += wj * x.y;
+          acc.z += wj * x.z;
+          acc.w += wj * x.w;
+        }
+      }
+      __syncthreads();
+    }
+    if (tr < nr) {
+      const int row = rb + tr;
+      const int i = row / p.Gc, hh = row % p.Gc;
+      if (hc * p.Gc + hh < p.G) {
+        const float L = row_s[RC + tr];
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const int h = g * p.G + hc * p.Gc + hh;
+        __nv_bfloat16* dst =
+            p.out + ((static_cast<long long>(b) * p.K + i) * p.Hq + h) * D + tq * 4;
+        uint2 pk;
+        pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+        pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+        *reinterpret_cast<uint2*>(dst) = pk;
+      }
+    }
+    __syncthreads();
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_splitkv_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -464,7 +609,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     const long long T = total_tiles(p, blockIdx.x == 0);
     long long a, b;
-    cta_range(p, T, gridDim.x, blockIdx.x, &a, &b);
+    OwnSeg own{-1, 0, 0, 0};
+    cta_range(p, T, gridDim.x, blockIdx.x, &a, &b, &own);
     Cursor c0{};
     if (b > a) cursor_seek(c0, p, a);
     sched[0] = a;
@@ -473,6 +619,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     sched[3] = (static_cast<long long>(c0.b) << 32) | static_cast<unsigned int>(c0.seg);
     sched[4] = (static_cast<long long>(c0.t) << 32) | static_cast<unsigned int>(c0.L);
     sched[5] = c0.nt;
+    sched[6] = own.s;
+    sched[7] = (static_cast<long long>(own.c0) << 32) | static_cast<unsigned int>(own.cn);
+    sched[8] = own.ns;
   }
 
   if (threadIdx.x == 0) {
@@ -935,10 +1084,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_dealloc(tmem, TMEM_COLS);
   }
 
+  const int RV = p.Gc * p.K;
+  if (sched[6] >= 0) {
+    // Per-segment partition: the cn CTAs of this CTA's segment each add to the
+    // segment's counter once their piece is written (the first adds 2^20 -
+    // (cn - 1), the rest 1, so every call adds exactly 2^20 and the counter
+    // never needs a reset); a CTA's own add pins the call's target.  Then the
+    // segment's rows are merged by its own CTAs, an equal share each.
+    const OwnSeg own{sched[6], static_cast<int>(sched[7] >> 32),
+                     static_cast<int>(sched[7] & 0xffffffff), static_cast<int>(sched[8])};
+    const int k = static_cast<int>(blockIdx.x) - own.c0;
+    const int row0 = static_cast<int>(mul_div(k, RV, own.cn));
+    const int row1 = static_cast<int>(mul_div(k + 1, RV, own.cn));
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned long long add = k == 0 ? (1ull << 20) - (own.cn - 1) : 1ull;
+      const unsigned long long old = atomicAdd(p.seg_cnt + own.s, add);
+      if (row1 > row0) grid_wait(p.seg_cnt + own.s, ((old >> 20) + 1) << 20, p.dev_status);
+    }
+    __syncthreads();
+    merge_segment<D>(p, own, row0, row1, warp, lane, smem + Ly::OFF_K, abort_flag);
+    return;
+  }
+
   // Every CTA's partials are written: meet at the grid barrier, then merge an
   // equal share of the output rows.  Thread 0 first records which CTAs hold
   // pieces of the segments of this CTA's rows (into the now idle K ring).
-  const int RV = p.Gc * p.K;
   const long long R = static_cast<long long>(p.B) * nseg * RV;
   const long long r0 = mul_div(blockIdx.x, R, gridDim.x);
   const long long r1 = mul_div(blockIdx.x + 1, R, gridDim.x);
@@ -978,15 +1149,21 @@ int check_shape(int B, int Hq, int Hkv, int d, int K, Shape* sh) {
   return ORTHRUS_OK;
 }
 
-// Workspace: [0, 256) grid-barrier words (must be zero before the first use;
-// every call leaves them zero), then the partial O and (m, l) of every piece.
-constexpr size_t WS_HEADER = 256;
+// Workspace: [0, 256) the grid-barrier ticket, then one 64-bit completion
+// counter per segment (padded to 256 bytes), then the partial O and (m, l) of
+// every piece.  The counters must be zero before the first use; every call
+// advances them by fixed amounts, so they never need resetting.
+constexpr size_t WS_TICKET = 256;
+
+size_t counter_bytes(const Shape& sh) {
+  return (static_cast<size_t>(sh.S) * sizeof(unsigned long long) + 255) / 256 * 256;
+}
 
 size_t workspace_bytes(const Shape& sh, int sms) {
   const size_t slots = static_cast<size_t>(sh.S) + static_cast<size_t>(sms);
   const size_t o_bytes = slots * ROWS * sh.d * sizeof(float);
   const size_t ml_bytes = slots * ROWS * sizeof(float2);
-  return WS_HEADER + o_bytes + ml_bytes;
+  return WS_TICKET + counter_bytes(sh) + o_bytes + ml_bytes;
 }
 
 template <int D>
@@ -1020,8 +1197,10 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   const size_t slots = static_cast<size_t>(sh.S) + static_cast<size_t>(sms);
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.gbar = reinterpret_cast<unsigned long long*>(w);
-  p.part_o = reinterpret_cast<float*>(w + WS_HEADER);
-  p.part_ml = reinterpret_cast<float2*>(w + WS_HEADER + slots * ROWS * D * sizeof(float));
+  p.seg_cnt = reinterpret_cast<unsigned long long*>(w + WS_TICKET);
+  const size_t head = WS_TICKET + counter_bytes(sh);
+  p.part_o = reinterpret_cast<float*>(w + head);
+  p.part_ml = reinterpret_cast<float2*>(w + head + slots * ROWS * D * sizeof(float));
   p.out = static_cast<__nv_bfloat16*>(out);
   p.dev_status = dev_status;
   p.B = sh.B;

@@ -65,6 +65,8 @@ ATTN_CASES = [
     (1, 16, 16, 2, 64, [300], None),               # G*K = 128 exactly
     (2, 32, 16, 2, 128, [100, 70], None),          # G*K = 256 -> two head chunks
     (1, 8, 4, 1, 64, [50], None),                  # one short segment: most CTAs idle
+    (1, 32, 8, 2, 128, [6000], None),              # 2 segments x 74 CTAs: merge in 2 batches
+    (1, 32, 12, 2, 64, [500], None),               # G = 6 over 4-head chunks: padding heads
     (20, 4, 16, 8, 64, list(range(60, 1260, 60)), None),  # 160 segments > 148 CTAs
 ]
 
@@ -137,9 +139,32 @@ def test_block_attn_repeat_calls_same_workspace_are_deterministic():
     b = ob.block_attn(q, kc, vc, cl, ob.MASK_AR, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
-    # the grid-barrier ticket counter advanced by exactly one grid per call
+    # 16 segments (2 sequences x 8 KV heads) <= SMs: each CTA works inside one
+    # segment, so the grid-barrier ticket is unused and each segment's
+    # completion counter (after the 256-byte ticket block) grew by 2^20 per call
+    head = ws[:256 + 16 * 8].view(torch.int64).cpu()
+    assert int(head[0]) == 0
+    assert head[32:48].tolist() == [2 << 20] * 16
+
+
+def test_block_attn_stream_k_mode_advances_the_grid_ticket():
+    # 20 sequences x 8 KV heads = 160 segments > 148 SMs: the flat tile range is
+    # split evenly and all CTAs meet at the grid barrier before the merge
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert int(ws[:8].view(torch.int64).item()) == 2 * sms
+    B = sms // 8 + 2
+    case = synth.attn_case(B, 4, 16, 8, 64, [60 + 7 * i for i in range(B)], seed=9)
+    q, kc, vc = case.q.cuda(), case.k_cache.cuda(), case.v_cache.cuda()
+    cl = torch.from_numpy(case.ctx_lens).cuda()
+    ws = torch.zeros(ob.block_attn_workspace_size(B, 16, 8, 64, 4), dtype=torch.uint8,
+                     device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for _ in range(3):
+        out = ob.block_attn(q, kc, vc, cl, ob.MASK_DIFF, workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert int(ws[:8].view(torch.int64).item()) == 3 * sms
+    ref = oracle.block_attn(case.q, case.k_cache, case.v_cache, case.ctx_lens, ob.MASK_DIFF)
+    assert_attn_close(out.cpu(), ref)
 
 
 def _check_argmax(got, ref_am, gap):
