@@ -65,6 +65,15 @@ typedef enum {
   ORTHRUS_MASK_AR = 1
 } orthrus_mask_mode;
 
+/* Option bit OR-ed into mask_mode of orthrus_block_attn (no counterpart in
+ * the method: an implementation choice).  By default the CTAs that share a
+ * (sequence, KV head) segment claim its last ~quarter of key groups
+ * dynamically, which balances their finish times but makes the fp32
+ * summation order, hence the last bits of the output, vary between calls.
+ * With this bit every CTA takes a fixed key range and repeated calls on the
+ * same inputs are bitwise identical. */
+#define ORTHRUS_ATTN_DETERMINISTIC 0x100
+
 /*
  * One layer's view of the shared KV cache ([GIST 2.1, 3]; [ABS]).
  *   k, v      bf16 [B, Hkv, cap, d] device.  Slots [0, ctx_lens[b]) hold the
@@ -113,13 +122,14 @@ int orthrus_block_attn_workspace_size(int B, int Hq, int Hkv, int d, int K, size
  *   q          bf16 [B, K, Hq, d] device (post-RoPE queries)
  *   cache      KV cache view (host struct; its pointers are device pointers)
  *   Hq, K      query heads (multiple of cache->Hkv), block size 1..32
- *   mask_mode  orthrus_mask_mode
+ *   mask_mode  orthrus_mask_mode, optionally | ORTHRUS_ATTN_DETERMINISTIC
  *   out        bf16 [B, K, Hq, d] device
  *   workspace  device, >= orthrus_block_attn_workspace_size(...) bytes, zero
  *              filled before the first call.  Its head holds a grid-barrier
- *              counter and one completion counter per (sequence, KV head, head
- *              chunk) segment; each call advances every counter it uses by a
- *              fixed amount, which keeps them consistent for the next call, so
+ *              counter and, per (sequence, KV head, head chunk) segment, a
+ *              completion counter and a work-claim counter; each call advances
+ *              them in a way the next call can rebase on (the completion
+ *              counters by exactly 2^20, the grid counter by the grid size), so
  *              a workspace is zeroed once, not per call (zero it again after an
  *              ORTHRUS_ETIMEOUT, and before using it on a device with a
  *              different SM count).  The rest holds per-call partial results.

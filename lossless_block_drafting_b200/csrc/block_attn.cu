@@ -60,6 +60,18 @@ constexpr int NSB = 2;
 constexpr int SBUF_COLS = 2 * TN;
 constexpr int TMEM_O = NSB * SBUF_COLS;  // O_0 at 256, O_1 at 384
 
+// The producer warp publishes the CTA's load groups, in order, as items of a
+// ring in shared memory: int4 {first tile | flags << 25, L of the sequence,
+// flat segment index, first cache row of the (sequence, KV head)}.
+constexpr int RING = 16;
+constexpr int kItemFlagShift = 25;
+constexpr int kItemTileMask = (1 << kItemFlagShift) - 1;
+constexpr int kItemPair = 1;        // two tiles (else one)
+constexpr int kItemPieceFirst = 2;  // first group of a piece (load its Q)
+constexpr int kItemPieceLast = 4;   // last group of a piece (publish its partial)
+constexpr int kItemEnd = 8;         // last group of the CTA
+constexpr int kItemNone = 16;       // the CTA has no group at all
+
 template <int D>
 struct Layout {
   static constexpr int CHUNKS = D / 64;            // 128-byte column chunks of a row
@@ -75,12 +87,16 @@ struct Layout {
   static constexpr int OFF_V = OFF_K + NK * KV_BYTES;
   static constexpr int OFF_ML = OFF_V + NV * KV_BYTES;  // [ROWS] float2 handed WG1 -> WG0
   static constexpr int OFF_SCHED = OFF_ML + ROWS * 8;  // 9 x int64 CTA schedule
-  static constexpr int OFF_BAR = OFF_SCHED + 128;
-  static constexpr int NBAR = 2 * NK + 2 * NV + 13;
+  static constexpr int OFF_ITEMS = OFF_SCHED + 128;  // RING x int4 work items
+  static constexpr int OFF_BAR = OFF_ITEMS + RING * 16;
+  static constexpr int NBAR = 2 * NK + 2 * NV + 13 + RING;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
 };
+
+static_assert(RING > Layout<64>::NK + NSB + 1 && RING > Layout<128>::NK + NSB + 1,
+              "work-item ring must outlast the pipeline depth");
 
 struct Params {
   const int32_t* ctx_lens;
@@ -88,9 +104,11 @@ struct Params {
   float2* part_ml;    // [slots][ROWS] (m in log2 units, l)
   unsigned long long* gbar;  // grid-barrier arrival ticket counter (starts at 0)
   unsigned long long* seg_cnt;  // [S] per-segment completion counters (start at 0)
+  unsigned long long* seg_next; // [S] per-segment group claim counters (start at 0)
   __nv_bfloat16* out; // [B, K, Hq, D]
   int32_t* dev_status;
   int B, K, Hq, Hkv, G, Gc, nhc, cap, mask_mode;
+  int balance;        // per-segment partition: claim the tail groups dynamically
   float sl2;          // softmax scale * log2(e)
 };
 
@@ -120,21 +138,6 @@ __device__ __forceinline__ void cursor_load(Cursor& c, const Params& p) {
   c.nt = n_tiles(c.L, p);
 }
 
-__device__ void cursor_seek(Cursor& c, const Params& p, long long x) {
-  const int nseg = p.Hkv * p.nhc;
-  c.b = 0;
-  c.base = 0;
-  cursor_load(c, p);
-  while (c.b + 1 < p.B && x >= c.base + static_cast<long long>(nseg) * c.nt) {
-    c.base += static_cast<long long>(nseg) * c.nt;
-    ++c.b;
-    cursor_load(c, p);
-  }
-  const long long local = x - c.base;
-  c.seg = static_cast<int>(mul_div(local, 1, c.nt));
-  c.t = static_cast<int>(local - static_cast<long long>(c.seg) * c.nt);
-}
-
 __device__ __forceinline__ void cursor_next(Cursor& c, const Params& p) {
   if (++c.t < c.nt) return;
   c.t = 0;
@@ -143,17 +146,6 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const Params& p) {
   c.seg = 0;
   c.base += static_cast<long long>(nseg) * c.nt;
   if (++c.b < p.B) cursor_load(c, p);
-}
-
-__device__ long long total_tiles(const Params& p, bool report_errors) {
-  long long T = 0;
-  const int nseg = p.Hkv * p.nhc;
-  for (int b = 0; b < p.B; ++b) {
-    const int raw = __ldg(p.ctx_lens + b);
-    if (report_errors && (raw < 0 || raw > p.cap - p.K)) report(p.dev_status, ORTHRUS_ECAPACITY);
-    T += static_cast<long long>(nseg) * n_tiles(clamp_len(raw, p), p);
-  }
-  return T;
 }
 
 // Load groups: a group starts at an even tile of a segment (or at the CTA's
@@ -173,37 +165,6 @@ __device__ __forceinline__ bool group_last(const Cursor& c, int j, int n) {
 // (pipeline drain, partial write, Q reload).  With more segments than CTAs
 // the flat tile range is split evenly (stream-K style) and a CTA may cross
 // segments.  Both kernels derive the same partition from ctx_lens.
-struct SegWalk {
-  int b, seg, ns;       // current segment (sequence b, KV head x head chunk seg), its tiles
-  long long Ts;         // first flat tile of the segment
-  int c0, cn;           // its CTAs [c0, c0 + cn)
-};
-
-template <typename F>
-__device__ __forceinline__ void walk_segments(const Params& p, long long T, int P, F&& f) {
-  const int nseg = p.Hkv * p.nhc;
-  const long long S = static_cast<long long>(p.B) * nseg;
-  long long sum_c = 0;
-  for (int b = 0; b < p.B; ++b) {
-    const int ns = n_tiles(clamp_len(__ldg(p.ctx_lens + b), p), p);
-    const long long extra = mul_div(static_cast<long long>(P) - S, ns, T);
-    for (int sg = 0; sg < nseg; ++sg) sum_c += 1 + extra;
-  }
-  const long long rem = P - sum_c;  // < S
-  long long Ts = 0, c0 = 0, si = 0;
-  for (int b = 0; b < p.B; ++b) {
-    const int ns = n_tiles(clamp_len(__ldg(p.ctx_lens + b), p), p);
-    const long long extra = mul_div(static_cast<long long>(P) - S, ns, T);
-    for (int sg = 0; sg < nseg; ++sg, ++si) {
-      const int cn = static_cast<int>(1 + extra + (si < rem ? 1 : 0));
-      SegWalk w{b, sg, ns, Ts, static_cast<int>(c0), cn};
-      if (f(w)) return;
-      Ts += ns;
-      c0 += cn;
-    }
-  }
-}
-
 __device__ __forceinline__ bool segment_partition(const Params& p, int P) {
   return static_cast<long long>(p.B) * p.Hkv * p.nhc <= P;
 }
@@ -217,30 +178,123 @@ __device__ __forceinline__ long long cta_of(long long x, long long T, long long 
   return mul_div((x + 1) * P - 1, 1, T);
 }
 
-// Flat tile range [x0, x1) of CTA c.  Under the per-segment partition *own
-// receives the CTA's segment (flat index, its CTAs and tiles).
+// Under the per-segment partition: the CTA's segment (flat index), its CTAs
+// [c0, c0 + cn), its tiles ns and the sequence's clamped context length L.
 struct OwnSeg {
   long long s;
-  int c0, cn, ns;
+  int c0, cn, ns, L;
 };
 
-__device__ void cta_range(const Params& p, long long T, int P, int c, long long* x0,
-                          long long* x1, OwnSeg* own) {
-  if (!segment_partition(p, P)) {
-    *x0 = cta_start(c, T, P);
-    *x1 = cta_start(c + 1, T, P);
-    return;
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+// Exclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ int warp_excl_scan(int v, int lane) {
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
   }
-  *x0 = *x1 = T;
+  return x - v;
+}
+
+// CTA c's work record, computed by the 32 lanes of one warp (sequences spread
+// over the lanes, running prefix sums by warp scans); the lane that owns CTA
+// c's sequence writes sched[0..8]:
+//   [0], [1]  flat tile range [x0, x1)
+//   [2]..[5]  the cursor at x0 (base, b | seg, t | L, nt)
+//   [6]..[8]  the CTA's segment under the per-segment partition (s, or -1;
+//             c0 | cn; L | ns)
+// Per-segment partition (S <= P): sequence b's segments get e_b = 1 +
+// floor((P - S) * n_b / T) CTAs each, the first P - sum of those segments one
+// more, and a CTA splits its segment's tiles evenly with its siblings.
+// Stream-K (S > P): the flat range of T tiles is split evenly.  All counts
+// fit in 32 bits (B * Hkv * cap < 2^31 is checked on the host).
+__device__ void warp_schedule(const Params& p, int P, int c, int lane, bool report_errors,
+                              long long* sched) {
   const int nseg = p.Hkv * p.nhc;
-  walk_segments(p, T, P, [&](const SegWalk& w) {
-    if (c < w.c0 || c >= w.c0 + w.cn) return false;
-    const long long k = c - w.c0;
-    *x0 = w.Ts + mul_div(k, w.ns, w.cn);
-    *x1 = w.Ts + mul_div(k + 1, w.ns, w.cn);
-    *own = OwnSeg{static_cast<long long>(w.b) * nseg + w.seg, w.c0, w.cn, w.ns};
-    return true;
-  });
+  const int S = p.B * nseg;
+  int tl = 0;
+  for (int b = lane; b < p.B; b += 32) {
+    const int raw = __ldg(p.ctx_lens + b);
+    if (report_errors && (raw < 0 || raw > p.cap - p.K)) report(p.dev_status, ORTHRUS_ECAPACITY);
+    tl += nseg * n_tiles(clamp_len(raw, p), p);
+  }
+  const int T = warp_sum(tl);
+  const bool segp = S <= P;
+  int rem = 0;
+  if (segp) {
+    int vl = 0;
+    for (int b = lane; b < p.B; b += 32)
+      vl += nseg * (1 + static_cast<int>(mul_div(P - S, n_tiles(clamp_len(__ldg(p.ctx_lens + b), p), p), T)));
+    rem = P - warp_sum(vl);  // < S
+  }
+  const int x0s = static_cast<int>(mul_div(c, T, P)), x1s = static_cast<int>(mul_div(c + 1, T, P));
+  bool found = false;
+  int Cb = 0, TTb = 0;  // CTAs and tiles of the sequences before this chunk
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    const bool in = b < p.B;
+    const int L = in ? clamp_len(__ldg(p.ctx_lens + b), p) : 0;
+    const int nb = in ? n_tiles(L, p) : 0;
+    const int e = in ? 1 + static_cast<int>(mul_div(P - S, nb, T)) : 0;
+    const int v = segp ? nseg * e : 0;
+    const int u = nseg * nb;
+    const int Cx = Cb + warp_excl_scan(v, lane), TTx = TTb + warp_excl_scan(u, lane);
+    if (in) {
+      int x0 = -1, x1 = 0, sg = 0, s_own = -1, c0 = 0, cn = 0;
+      if (segp) {
+        const int bs = b * nseg;
+        const int lo = Cx + min(bs, rem);
+        const int hi = Cx + v + min(bs + nseg, rem);
+        if (c >= lo && c < hi) {
+          const int rb = max(0, min(nseg, rem - bs));  // segments of b with one more CTA
+          const int local = c - lo;
+          int k;
+          if (local < rb * (e + 1)) {
+            sg = local / (e + 1);
+            k = local - sg * (e + 1);
+            cn = e + 1;
+          } else {
+            const int l2 = local - rb * (e + 1);
+            sg = rb + l2 / e;
+            k = l2 - (sg - rb) * e;
+            cn = e;
+          }
+          const int Ts = TTx + sg * nb;
+          x0 = Ts + static_cast<int>(mul_div(k, nb, cn));
+          x1 = Ts + static_cast<int>(mul_div(k + 1, nb, cn));
+          s_own = bs + sg;
+          c0 = c - k;
+        }
+      } else if (x1s > x0s && x0s >= TTx && x0s < TTx + u) {
+        sg = (x0s - TTx) / nb;
+        x0 = x0s;
+        x1 = x1s;
+      }
+      if (x0 >= 0) {
+        found = true;
+        sched[0] = x0;
+        sched[1] = x1;
+        sched[2] = TTx;
+        sched[3] = (static_cast<long long>(b) << 32) | static_cast<unsigned int>(sg);
+        sched[4] = (static_cast<long long>(x0 - TTx - sg * nb) << 32) | static_cast<unsigned int>(L);
+        sched[5] = nb;
+        sched[6] = s_own;
+        sched[7] = (static_cast<long long>(c0) << 32) | static_cast<unsigned int>(cn);
+        sched[8] = (static_cast<long long>(L) << 32) | static_cast<unsigned int>(nb);
+      }
+    }
+    Cb += warp_sum(v);
+    TTb += warp_sum(u);
+  }
+  if (!__any_sync(0xFFFFFFFFu, found) && lane == 0) {  // no tiles for this CTA
+    for (int i = 0; i < 9; ++i) sched[i] = 0;
+    sched[6] = -1;
+  }
 }
 
 // Wait that ignores the abort flag, used only to drain in-flight async work
@@ -297,21 +351,9 @@ __device__ void segment_ctas(const Params& p, int P, int b, int seg, long long* 
     T += static_cast<long long>(nseg) * nt;
   }
   *ntb = nt_b;
-  if (segment_partition(p, P)) {
-    *c0 = 0;
-    *c1 = -1;
-    walk_segments(p, T, P, [&](const SegWalk& w) {
-      if (w.b != b || w.seg != seg) return false;
-      *c0 = w.c0;
-      *c1 = w.c0 + w.cn - 1;
-      return true;
-    });
-    *tall = -1;
-  } else {
-    *c0 = cta_of(Ts, T, P);
-    *c1 = cta_of(Ts + nt_b - 1, T, P);
-    *tall = T;
-  }
+  *c0 = cta_of(Ts, T, P);
+  *c1 = cta_of(Ts + nt_b - 1, T, P);
+  *tall = T;
 }
 
 // Pieces of one segment, as seen by the merge: CTAs [c0, c1]; when `dense`
@@ -457,7 +499,8 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
     fence_mbar_init();
   }
   __syncthreads();
-  const bool dense = own.cn <= own.ns;  // every CTA of the segment wrote a piece
+  // every CTA of the segment wrote a piece (or, balanced, an empty one)
+  const bool dense = p.balance || own.cn <= own.ns;
   auto live = [&](int j) {
     return dense || mul_div(j, own.ns, own.cn) != mul_div(j + 1, own.ns, own.cn);
   };
@@ -599,6 +642,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t o_full = bar2 + 8u * 10;
   const uint32_t o_free = bar2 + 8u * 11;
   const uint32_t mma_done = bar2 + 8u * 12;  // both MMA issuers commit once at exit
+  auto item_full = [&](int i) { return bar2 + 8u * (13 + i); };  // work item i published
+  int4* items = reinterpret_cast<int4*>(smem + Ly::OFF_ITEMS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
   float2* ml_xchg = reinterpret_cast<float2*>(smem + Ly::OFF_ML);
@@ -606,23 +651,159 @@ __global__ void __launch_bounds__(THREADS, 1)
   // The CTA's tile range and its starting cursor are computed once, by
   // thread 0, and shared.
   long long* sched = reinterpret_cast<long long*>(smem + Ly::OFF_SCHED);
-  if (threadIdx.x == 0) {
-    const long long T = total_tiles(p, blockIdx.x == 0);
-    long long a, b;
-    OwnSeg own{-1, 0, 0, 0};
-    cta_range(p, T, gridDim.x, blockIdx.x, &a, &b, &own);
-    Cursor c0{};
-    if (b > a) cursor_seek(c0, p, a);
-    sched[0] = a;
-    sched[1] = b;
-    sched[2] = c0.base;
-    sched[3] = (static_cast<long long>(c0.b) << 32) | static_cast<unsigned int>(c0.seg);
-    sched[4] = (static_cast<long long>(c0.t) << 32) | static_cast<unsigned int>(c0.L);
-    sched[5] = c0.nt;
-    sched[6] = own.s;
-    sched[7] = (static_cast<long long>(own.c0) << 32) | static_cast<unsigned int>(own.cn);
-    sched[8] = own.ns;
+  if (warp == 0) {
+    warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
+    __syncwarp();
   }
+
+  const int nseg = p.Hkv * p.nhc;
+  // Per-segment partition: this CTA's segment (s = -1 in stream-K mode),
+  // read where it is needed rather than kept live through the tile loops.
+  auto read_own = [&]() {
+    const volatile long long* sv = sched;
+    return OwnSeg{sv[6], static_cast<int>(sv[7] >> 32), static_cast<int>(sv[7] & 0xffffffff),
+                  static_cast<int>(sv[8] & 0xffffffff), static_cast<int>(sv[8] >> 32)};
+  };
+  auto read_start = [&]() {
+    Cursor c;
+    c.base = sched[2];
+    c.b = static_cast<int>(sched[3] >> 32);
+    c.seg = static_cast<int>(sched[3] & 0xffffffff);
+    c.t = static_cast<int>(sched[4] >> 32);
+    c.L = static_cast<int>(sched[4] & 0xffffffff);
+    c.nt = static_cast<int>(sched[5]);
+    return c;
+  };
+
+  // ---------------------------------------- work list, Q and K producer
+  // Thread 0 decides the CTA's load groups (up to two 64-key tiles of one
+  // segment), publishes each as an item of the shared ring (every other role
+  // replays the same list) and issues the Q tile of each piece and the
+  // group's K.  produce(limit) emits groups until `limit` have been emitted
+  // or the list ends; it runs once before the prologue barrier (the first NK
+  // groups need no free stage, so HBM traffic starts right after the
+  // schedule) and resumes in the producer role.
+  int pr_gi = 0, pr_pieces = 0;
+  OwnSeg pr_own{-1, 0, 0, 0, 0};
+  Cursor pr_c{};
+  int pr_n = 0, pr_j = 0, pr_cur = -2;
+  int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0, pr_have = 0, pr_bnext = 0;
+  bool pr_grabbing = false, pr_dry = true;
+  unsigned long long pr_base = 0, pr_pend = 0;
+  const uint64_t pr_policy = policy_evict_first();
+  auto emit = [&](int t, int L, long long s, int flags) -> bool {
+    const int slot = pr_gi % RING;
+    const int b = static_cast<int>(s / nseg), seg = static_cast<int>(s % nseg);
+    const int g = seg / p.nhc, hc = seg % p.nhc;
+    const int kvbase = (b * p.Hkv + g) * p.cap;
+    // Ring slots are never overwritten early: the producer is at most NK
+    // groups ahead of S = Q K^T, which is at most NSB groups ahead of P V,
+    // which trails every other reader of an item (RING > NK + NSB + 1).
+    items[slot] = make_int4(t | (flags << kItemFlagShift), L, static_cast<int>(s), kvbase);
+    mbar_arrive(item_full(slot));
+    if (flags & kItemNone) return true;
+    if (flags & kItemPieceFirst) {
+      if (!mbar_wait_bounded(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status)) return false;
+      mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.Gc * p.K * D * 2));
+      for (int c = 0; c < Ly::CHUNKS; ++c)
+        tma_load_3d(sb0 + Ly::OFF_Q + c * Ly::Q_CHUNK, &tmQ, q_full, c * 64,
+                    g * p.G + hc * p.Gc, b * p.K);
+      ++pr_pieces;
+    }
+    const bool pair = flags & kItemPair;
+    const int stage = pr_gi % NK;
+    if (!mbar_wait_bounded(empty_k(stage), ((pr_gi / NK) & 1) ^ 1, abort_flag, p.dev_status))
+      return false;
+    mbar_arrive_expect_tx(full_k(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
+    for (int c = 0; c < Ly::CHUNKS; ++c)
+      tma_load_2d_hint(sb0 + Ly::OFF_K + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
+                       pair ? &tmK2 : &tmK1, full_k(stage), c * 64, kvbase + t * TN, pr_policy);
+    ++pr_gi;
+    return true;
+  };
+  // Balanced per-segment partition: the CTA first streams a static run of
+  // about 3/4 of its fair share of the segment's 128-key groups, then claims
+  // groups of the remaining pool two at a time from the segment's claim
+  // counter (one claim kept in flight, so its latency is hidden).  The
+  // counter is rebased per call to epoch E << 32, E being the number of
+  // completed calls read from the segment's completion counter (which cannot
+  // reach the next multiple of 2^20 before this CTA's own add).
+  auto start_claims = [&]() {
+    const unsigned long long done =
+        *reinterpret_cast<volatile unsigned long long*>(p.seg_cnt + pr_own.s);
+    pr_base = (done >> 20) << 32;
+    atomicMax(p.seg_next + pr_own.s, pr_base);
+    pr_pend = atomicAdd(p.seg_next + pr_own.s, 2ull);
+    pr_grabbing = true;
+  };
+  auto next_group = [&]() -> int {
+    if (pr_sg < pr_sg_end) {
+      const int g = pr_sg++;
+      if (!pr_grabbing && !pr_dry && pr_sg_end - pr_sg <= 1) start_claims();
+      return g;
+    }
+    if (pr_dry) return -1;
+    if (!pr_grabbing) start_claims();
+    if (pr_have == 0) {
+      const long long first = pr_pool0 + static_cast<long long>(pr_pend - pr_base);
+      if (first >= pr_ngr) {
+        pr_dry = true;
+        return -1;
+      }
+      pr_bnext = static_cast<int>(first);
+      pr_have = 2;
+      pr_pend = atomicAdd(p.seg_next + pr_own.s, 2ull);  // next claim, in flight
+    }
+    --pr_have;
+    if (pr_bnext >= pr_ngr) {
+      pr_dry = true;
+      return -1;
+    }
+    return pr_bnext++;
+  };
+  // Before the barrier (pre) no other role runs yet, so only groups that need
+  // no wait are emitted: the first NK (fresh K stages) of the first piece.
+  auto produce = [&](int limit, bool pre) {
+    if (pr_own.s >= 0 && p.balance) {
+      if (pr_cur == -2) {
+        pr_cur = next_group();
+        if (pr_cur < 0) emit(0, pr_own.L, pr_own.s, kItemNone);
+      }
+      while (pr_cur >= 0 && pr_gi < limit) {
+        const int nxt = next_group();
+        const bool pair = 2 * pr_cur + 1 < pr_own.ns;
+        const int flags = (pair ? kItemPair : 0) | (pr_gi == 0 ? kItemPieceFirst : 0) |
+                          (nxt < 0 ? (kItemPieceLast | kItemEnd) : 0);
+        if (!emit(2 * pr_cur, pr_own.L, pr_own.s, flags)) {
+          pr_cur = -1;
+          break;
+        }
+        pr_cur = nxt;
+      }
+    } else {
+      // Static range [x0, x0 + n) of the flat tile space (deterministic).
+      if (pr_cur == -2) {
+        pr_cur = 0;
+        if (pr_n == 0) emit(0, 0, pr_own.s, kItemNone);
+      }
+      while (pr_j < pr_n && pr_gi < limit) {
+        const bool pair = !group_last(pr_c, pr_j, pr_n);
+        const int jl = pr_j + (pair ? 1 : 0);
+        const bool pfirst = (pr_j == 0) || pr_c.t == 0;
+        const bool plast = (jl == pr_n - 1) || pr_c.t + (pair ? 1 : 0) == pr_c.nt - 1;
+        const int flags = (pair ? kItemPair : 0) | (pfirst ? kItemPieceFirst : 0) |
+                          (plast ? kItemPieceLast : 0) | (jl == pr_n - 1 ? kItemEnd : 0);
+        if (pre && pfirst && pr_pieces > 0) break;  // its Q waits for the previous piece's
+        if (!emit(pr_c.t, pr_c.L, static_cast<long long>(pr_c.b) * nseg + pr_c.seg, flags)) {
+          pr_j = pr_n;
+          break;
+        }
+        cursor_next(pr_c, p);
+        if (pair) cursor_next(pr_c, p);
+        pr_j = jl + 1;
+      }
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -644,8 +825,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(o_full, 1);
     mbar_init(o_free, 4);
     mbar_init(mma_done, 2);
+    for (int i = 0; i < RING; ++i) mbar_init(item_full(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // warp 0 wrote the schedule (the warp converged after warp_schedule)
+    pr_own = read_own();
+    pr_c = read_start();
+    pr_n = static_cast<int>(sched[1] - sched[0]);
+    if (pr_own.s >= 0 && p.balance) {
+      const int k = static_cast<int>(blockIdx.x) - pr_own.c0;
+      pr_ngr = (pr_own.ns + 1) / 2;
+      const int fs = static_cast<int>(mul_div(3 * pr_ngr, 1, 4 * pr_own.cn));
+      pr_pool0 = pr_own.cn * fs;
+      pr_sg = k * fs;
+      pr_sg_end = pr_sg + fs;
+      pr_dry = pr_pool0 >= pr_ngr;
+    }
+    produce(NK, true);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -668,86 +864,46 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const long long x0 = sched[0];
-  const int n = static_cast<int>(sched[1] - sched[0]);
-  Cursor start;
-  start.base = sched[2];
-  start.b = static_cast<int>(sched[3] >> 32);
-  start.seg = static_cast<int>(sched[3] & 0xffffffff);
-  start.t = static_cast<int>(sched[4] >> 32);
-  start.L = static_cast<int>(sched[4] & 0xffffffff);
-  start.nt = static_cast<int>(sched[5]);
-  const int nseg = p.Hkv * p.nhc;
 
 #define WAIT_OR(barrier, parity, on_fail) \
   if (!mbar_wait_bounded((barrier), (parity), abort_flag, p.dev_status)) on_fail
 #define WARP_WAIT_OR(barrier, parity, on_fail) \
   if (!mbar_wait_warp((barrier), (parity), abort_flag, p.dev_status)) on_fail
 
-  if (n > 0 && warp == 0 && lane == 0) {
-    // ------------------------------------------------- Q and K producer
-    prefetch_tmap(&tmQ);
-    prefetch_tmap(&tmK2);
-    prefetch_tmap(&tmK1);
-    const uint64_t policy = policy_evict_first();
-    Cursor cur;
-    cur = start;
-    int pieces = 0, gi = 0;
-    const uint32_t q_tx = static_cast<uint32_t>(p.Gc * p.K * D * 2);
-    for (int j = 0; j < n; ++j) {
-      const bool first = (j == 0) || cur.t == 0;
-      const int g = cur.seg / p.nhc, hc = cur.seg % p.nhc;
-      if (first) {
-        WAIT_OR(q_empty, (pieces & 1) ^ 1, break);
-        mbar_arrive_expect_tx(q_full, q_tx);
-        for (int c = 0; c < Ly::CHUNKS; ++c)
-          tma_load_3d(sb0 + Ly::OFF_Q + c * Ly::Q_CHUNK, &tmQ, q_full, c * 64,
-                      g * p.G + hc * p.Gc, cur.b * p.K);
-        ++pieces;
-      }
-      if (group_first(cur, j)) {
-        const bool pair = !group_last(cur, j, n);
-        const int stage = gi % NK;
-        const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
-        WAIT_OR(empty_k(stage), ((gi / NK) & 1) ^ 1, break);
-        mbar_arrive_expect_tx(full_k(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
-        for (int c = 0; c < Ly::CHUNKS; ++c)
-          tma_load_2d_hint(sb0 + Ly::OFF_K + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
-                           pair ? &tmK2 : &tmK1, full_k(stage), c * 64, row0, policy);
-        ++gi;
-      }
-      cursor_next(cur, p);
-    }
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------ work list, Q and K producer
+    // (its first NK groups were issued before the prologue barrier)
+    produce(1 << 30, false);
     // Drain: every issued copy must have landed before the CTA may exit.
-    for (int q = (gi > NK ? gi - NK : 0); q < gi; ++q)
+    for (int q = (pr_gi > NK ? pr_gi - NK : 0); q < pr_gi; ++q)
       mbar_wait_drain(full_k(q % NK), (q / NK) & 1, p.dev_status);
-    if (pieces > 0) mbar_wait_drain(q_full, (pieces - 1) & 1, p.dev_status);
-  } else if (n > 0 && warp == 2 && lane == 0) {
+    if (pr_pieces > 0) mbar_wait_drain(q_full, (pr_pieces - 1) & 1, p.dev_status);
+  } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------- V producer
     prefetch_tmap(&tmV2);
     prefetch_tmap(&tmV1);
     const uint64_t policy = policy_evict_first();
-    Cursor cur;
-    cur = start;
     int gi = 0;
-    for (int j = 0; j < n; ++j) {
-      if (group_first(cur, j)) {
-        const bool pair = !group_last(cur, j, n);
-        const int g = cur.seg / p.nhc;
-        const int stage = gi % NV;
-        const int row0 = (cur.b * p.Hkv + g) * p.cap + cur.t * TN;
-        WAIT_OR(empty_v(stage), ((gi / NV) & 1) ^ 1, break);
-        mbar_arrive_expect_tx(full_v(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
-        for (int c = 0; c < Ly::CHUNKS; ++c)
-          tma_load_2d_hint(sb0 + Ly::OFF_V + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
-                           pair ? &tmV2 : &tmV1, full_v(stage), c * 64, row0, policy);
-        ++gi;
-      }
-      cursor_next(cur, p);
+    for (;;) {
+      const int slot = gi % RING;
+      WAIT_OR(item_full(slot), (gi / RING) & 1, break);
+      const int4 it = items[slot];
+      const int flags = it.x >> kItemFlagShift;
+      if (flags & kItemNone) break;
+      const int t = it.x & kItemTileMask;
+      const bool pair = flags & kItemPair;
+      const int stage = gi % NV;
+      WAIT_OR(empty_v(stage), ((gi / NV) & 1) ^ 1, break);
+      mbar_arrive_expect_tx(full_v(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
+      for (int c = 0; c < Ly::CHUNKS; ++c)
+        tma_load_2d_hint(sb0 + Ly::OFF_V + stage * Ly::KV_BYTES + c * Ly::KV_CHUNK,
+                         pair ? &tmV2 : &tmV1, full_v(stage), c * 64, it.w + t * TN, policy);
+      ++gi;
+      if (flags & kItemEnd) break;
     }
     for (int q = (gi > NV ? gi - NV : 0); q < gi; ++q)
       mbar_wait_drain(full_v(q % NV), (q / NV) & 1, p.dev_status);
-  } else if (n > 0 && warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------ S = Q K^T issuer
     // One N = 128 (or 64 for a lone tile) MMA sequence per load group into
     // TMEM buffer g % 2; the buffer is reused once P*V of group g - 2 is done.
@@ -762,42 +918,39 @@ __global__ void __launch_bounds__(THREADS, 1)
       kd[kk] = make_sdesc(sb0 + Ly::OFF_K + (kk >> 2) * Ly::KV_CHUNK + (kk & 3) * 32, 16, 1024,
                           kSwizzle128B);
     }
-    Cursor cs;
-    cs = start;
     int q_seen = 0, gi = 0;
-    for (int j = 0; j < n; ++j) {
-      const bool first = (j == 0) || cs.t == 0;
-      const bool last = (j == n - 1) || cs.t == cs.nt - 1;
-      if (first) {
+    for (;;) {
+      const int slot = gi % RING;
+      WAIT_OR(item_full(slot), (gi / RING) & 1, break);
+      const int flags = items[slot].x >> kItemFlagShift;
+      if (flags & kItemNone) break;
+      if (flags & kItemPieceFirst) {
         WAIT_OR(q_full, q_seen & 1, break);
         ++q_seen;
       }
-      const bool glast = group_last(cs, j, n);
-      if (group_first(cs, j)) {
-        const int stage = gi % NK;
-        const int gb = gi & 1;
-        WAIT_OR(full_k(stage), (gi / NK) & 1, break);
-        if (gi >= NSB) {
-          WAIT_OR(sb_free(gb), ((gi >> 1) - 1) & 1, break);
-        }
-        tc_fence_after();
-        const uint64_t koff = static_cast<uint64_t>((stage * Ly::KV_BYTES) >> 4);
-        const uint32_t id = glast ? id_s1 : id_s2;
-        const uint32_t dst = tmem + gb * SBUF_COLS;
-        mma_bf16_ss(dst, qd[0], kd[0] + koff, id, 0u);
-#pragma unroll
-        for (int kk = 1; kk < D / 16; ++kk) mma_bf16_ss(dst, qd[kk], kd[kk] + koff, id, 1u);
-        mma_commit(empty_k(stage));
-        mma_commit(s_full(gb));
+      const int stage = gi % NK;
+      const int gb = gi & 1;
+      WAIT_OR(full_k(stage), (gi / NK) & 1, break);
+      if (gi >= NSB) {
+        WAIT_OR(sb_free(gb), ((gi >> 1) - 1) & 1, break);
       }
-      if (last) mma_commit(q_empty);
-      if (glast) ++gi;
-      cursor_next(cs, p);
+      tc_fence_after();
+      const uint64_t koff = static_cast<uint64_t>((stage * Ly::KV_BYTES) >> 4);
+      const uint32_t id = (flags & kItemPair) ? id_s2 : id_s1;
+      const uint32_t dst = tmem + gb * SBUF_COLS;
+      mma_bf16_ss(dst, qd[0], kd[0] + koff, id, 0u);
+#pragma unroll
+      for (int kk = 1; kk < D / 16; ++kk) mma_bf16_ss(dst, qd[kk], kd[kk] + koff, id, 1u);
+      mma_commit(empty_k(stage));
+      mma_commit(s_full(gb));
+      if (flags & kItemPieceLast) mma_commit(q_empty);
+      ++gi;
+      if (flags & kItemEnd) break;
     }
     // every MMA of both issuers must be complete before TMEM is released
     mma_commit(mma_done);
     mbar_wait_drain(mma_done, 0, p.dev_status);
-  } else if (n > 0 && warp == 3 && lane == 0) {
+  } else if (warp == 3 && lane == 0) {
     // ------------------------------------------------ O_w += P V issuer
     const uint32_t id_pv = make_idesc_bf16_f32(ROWS, D, false, true);
     uint64_t vd[TN / 16];
@@ -806,51 +959,53 @@ __global__ void __launch_bounds__(THREADS, 1)
       // V is [keys x d] with d contiguous: MN-major B operand; 16 keys per step
       // = two 8-row swizzle atoms (2048 B); d chunks Ly::KV_CHUNK apart.
       vd[kk] = make_sdesc(sb0 + Ly::OFF_V + kk * 2048, Ly::KV_CHUNK, 1024, kSwizzle128B);
-    Cursor cp;
-    cp = start;
-    int pieces_done = 0, jp = 0, gi = 0;
+    int pieces_done = 0, jp = 0, gi = 0, j = 0;
     int pf_uses[2 * NSB] = {0, 0, 0, 0};  // completed phases seen per P barrier
-    for (int j = 0; j < n; ++j) {
-      const bool first = (j == 0) || cp.t == 0;
-      const bool last = (j == n - 1) || cp.t == cp.nt - 1;
-      if (first) {
+    bool fail = false;
+    for (;;) {
+      const int slot = gi % RING;
+      WAIT_OR(item_full(slot), (gi / RING) & 1, break);
+      const int flags = items[slot].x >> kItemFlagShift;
+      if (flags & kItemNone) break;
+      if (flags & kItemPieceFirst) {
         jp = j;
         if (pieces_done > 0) {
           WAIT_OR(o_free, (pieces_done - 1) & 1, break);
         }
       }
-      const int w = j & 1;
-      const bool gfirst = group_first(cp, j), glast = group_last(cp, j, n);
-      const int gb = gi & 1, half = gfirst ? 0 : 1;
-      const int pb = 2 * gb + half;
-      WAIT_OR(p_full(pb), pf_uses[pb] & 1, break);
-      ++pf_uses[pb];
-      const int stage = gi % NV;
-      if (gfirst) {
-        WAIT_OR(full_v(stage), (gi / NV) & 1, break);
-      }
-      tc_fence_after();
-      const uint64_t voff = static_cast<uint64_t>((stage * Ly::KV_BYTES + half * Ly::HALF) >> 4);
-      const uint32_t a_p = tmem + gb * SBUF_COLS + half * TN;  // P: 16 keys = 8 columns
-      const uint32_t dst = tmem + TMEM_O + w * 128;
-      const bool fresh = (j - jp) < 2;  // first tile of group w in this piece
-      mma_bf16_ts(dst, a_p, vd[0] + voff, id_pv, fresh ? 0u : 1u);
+      const int gb = gi & 1, stage = gi % NV;
+      const int ntl = (flags & kItemPair) ? 2 : 1;
+      for (int h = 0; h < ntl; ++h, ++j) {
+        const int w = j & 1;
+        const int pb = 2 * gb + h;
+        WAIT_OR(p_full(pb), pf_uses[pb] & 1, { fail = true; break; });
+        ++pf_uses[pb];
+        if (h == 0) {
+          WAIT_OR(full_v(stage), (gi / NV) & 1, { fail = true; break; });
+        }
+        tc_fence_after();
+        const uint64_t voff = static_cast<uint64_t>((stage * Ly::KV_BYTES + h * Ly::HALF) >> 4);
+        const uint32_t a_p = tmem + gb * SBUF_COLS + h * TN;  // P: 16 keys = 8 columns
+        const uint32_t dst = tmem + TMEM_O + w * 128;
+        const bool fresh = (j - jp) < 2;  // first tile of group w in this piece
+        mma_bf16_ts(dst, a_p, vd[0] + voff, id_pv, fresh ? 0u : 1u);
 #pragma unroll
-      for (int kk = 1; kk < TN / 16; ++kk) mma_bf16_ts(dst, a_p + kk * 8, vd[kk] + voff, id_pv, 1u);
-      if (glast) {
-        mma_commit(empty_v(stage));
-        mma_commit(sb_free(gb));
-        ++gi;
+        for (int kk = 1; kk < TN / 16; ++kk)
+          mma_bf16_ts(dst, a_p + kk * 8, vd[kk] + voff, id_pv, 1u);
       }
-      if (last) {
+      if (fail) break;
+      mma_commit(empty_v(stage));
+      mma_commit(sb_free(gb));
+      if (flags & kItemPieceLast) {
         mma_commit(o_full);
         ++pieces_done;
       }
-      cursor_next(cp, p);
+      ++gi;
+      if (flags & kItemEnd) break;
     }
     mma_commit(mma_done);
     mbar_wait_drain(mma_done, 0, p.dev_status);
-  } else if (n > 0 && warp >= 4) {
+  } else if (warp >= 4) {
     // ------------------------------------------------ softmax + epilogue
     const int w = (warp - 4) >> 2;            // softmax warpgroup: even / odd tiles
     const int r = (warp & 3) * 32 + lane;     // query row == TMEM lane
@@ -860,10 +1015,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int i_row = r / p.Gc;
     const bool idle_warp = (warp & 3) * 32 >= rows_valid;
     const float sl2 = p.sl2;
-    Cursor cur;
-    cur = start;
-    int pieces = 0, jp = 0, gi = 0, prev_gi = 0;
+    int pieces = 0, jp = 0, gi = 0, j = 0, prev_gi = 0;
     float m_used = -INFINITY, l_sum = 0.f;
+    bool fail = false;
+#define FAIL          \
+  {                   \
+    fail = true;      \
+    break;            \
+  }
     // A tile that runs past the valid keys: the warpgroup's 128 threads zero
     // those V rows together, so that stale or NaN cache contents cannot reach
     // O through 0 * NaN.  Returns false if the V stage never arrived.
@@ -881,45 +1040,65 @@ __global__ void __launch_bounds__(THREADS, 1)
       fence_proxy_async_smem();
       return true;
     };
-    for (int j = 0; j < n; ++j) {
-      const bool first = (j == 0) || cur.t == 0;
-      const bool last = (j == n - 1) || cur.t == cur.nt - 1;
-      if (first) {
+    for (;;) {
+      const int slot = gi % RING;
+      WARP_WAIT_OR(item_full(slot), (gi / RING) & 1, break);
+      const int2 itxy = *reinterpret_cast<const int2*>(&items[slot]);
+      const int flags = itxy.x >> kItemFlagShift;
+      if (flags & kItemNone) {
+        // No group at all: publish an empty piece (its m = -inf) for the merge.
+        const int s_it = items[slot].z;
+        if (w == 0 && s_it >= 0 && r < rows_valid)
+          p.part_ml[(static_cast<long long>(s_it) + blockIdx.x) * ROWS + r] =
+              make_float2(-INFINITY, 0.f);
+        break;
+      }
+      const int t0 = itxy.x & kItemTileMask;
+      const int Lc = itxy.y;
+      const int ntl = (flags & kItemPair) ? 2 : 1;
+      if (flags & kItemPieceFirst) {
         jp = j;
         m_used = -INFINITY;
         l_sum = 0.f;
       }
-      if ((j & 1) == w && idle_warp) {
-        // All 32 rows of this warp are padding: no softmax, but it still
-        // waits for S (which keeps it within one phase of the P barriers),
-        // takes its share of a tail tile's V zeroing, and arrives so the P*V
-        // issuer's count is complete.  The P rows it leaves unwritten feed
-        // only padding rows of O, which are never read.
-        WARP_WAIT_OR(s_full(gi & 1), (gi >> 1) & 1, break);
-        const int tile0 = cur.t * TN;
-        const int kv_end = cur.L + p.K;
-        if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, group_first(cur, j))) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(p_full(2 * (gi & 1) + (group_first(cur, j) ? 0 : 1)));
-        prev_gi = gi;
-      } else if ((j & 1) == w) {
-        const bool fresh = (j - jp) < 2;
+      // Tile h of the group is tile j + h of the CTA; warpgroup w takes the
+      // tiles with (j + h) & 1 == w: at most one per group.
+      const int h = (w - j) & 1;
+      const int jt = j + h;
+      j += ntl;
+      if (h < ntl) do {
+        if (idle_warp) {
+          // All 32 rows of this warp are padding: no softmax, but it still
+          // waits for S (which keeps it within one phase of the P barriers),
+          // takes its share of a tail tile's V zeroing, and arrives so the P*V
+          // issuer's count is complete.  The P rows it leaves unwritten feed
+          // only padding rows of O, which are never read.
+          WARP_WAIT_OR(s_full(gi & 1), (gi >> 1) & 1, FAIL);
+          const int tile0 = (t0 + h) * TN;
+          const int kv_end = Lc + p.K;
+          if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, h == 0)) FAIL;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(p_full(2 * (gi & 1) + h));
+          prev_gi = gi;
+          break;
+        }
+        const bool fresh = (jt - jp) < 2;
         const int gb = gi & 1;
-        const int half = group_first(cur, j) ? 0 : 1;
+        const int half = h;
         const uint32_t t_s = lane_base + gb * SBUF_COLS + half * TN;
-        const int kv_end = cur.L + p.K;
-        const int tile0 = cur.t * TN;
-        WARP_WAIT_OR(s_full(gb), (gi >> 1) & 1, break);
+        const int kv_end = Lc + p.K;
+        const int tile0 = (t0 + h) * TN;
+        WARP_WAIT_OR(s_full(gb), (gi >> 1) & 1, FAIL);
         tc_fence_after();
         uint32_t sr[TN];
         tmem_ld64(t_s, sr);
         tmem_wait_ld();
 
-        if (tile0 + TN > cur.L + 1) {
+        if (tile0 + TN > Lc + 1) {
           // Tail tile: some keys lie past some row's limit.  Interior tiles
           // (every key < L + 1) skip this entirely.
           const int lim = (r >= rows_valid) ? 0
-                          : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+                          : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : Lc + i_row + 1);
 #pragma unroll
           for (int c = 0; c < TN; ++c)
             if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
@@ -976,9 +1155,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             // tile max, rescale O_w and l, and redo the tile.
             tmem_ld64(t_s, sr);
             tmem_wait_ld();
-            if (tile0 + TN > cur.L + 1) {
+            if (tile0 + TN > Lc + 1) {
               const int lim = (r >= rows_valid) ? 0
-                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : cur.L + i_row + 1);
+                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : Lc + i_row + 1);
 #pragma unroll
               for (int c = 0; c < TN; ++c)
                 if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
@@ -996,16 +1175,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                             : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
             // O_w may only be touched once this group's previous P*V (tile
             // j - 2, in load group prev_gi) has completed.
-            WARP_WAIT_OR(sb_free(prev_gi & 1), (prev_gi >> 1) & 1, break);
+            WARP_WAIT_OR(sb_free(prev_gi & 1), (prev_gi >> 1) & 1, FAIL);
             tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(t_o + c0, o);
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(t_o + c0, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-              tmem_st32(t_o + c0, o);
+              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+              tmem_st16(t_o + c0, o);
             }
             tmem_wait_st();
             l_sum *= f;
@@ -1016,7 +1195,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float2 t2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
         l_sum += t2.x + t2.y;
 
-        if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, group_first(cur, j))) break;
+        if (tile0 + TN > kv_end && !zero_v_tail(tile0, kv_end, h == 0)) FAIL;
         uint32_t pk[TN / 2];
 #pragma unroll
         for (int c = 0; c < TN / 2; ++c) pk[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
@@ -1026,9 +1205,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(p_full(2 * gb + half));
         prev_gi = gi;
-      }
+      } while (0);
+      if (fail) break;
 
-      if (last) {
+      if (flags & kItemPieceLast) {
         // Piece epilogue: merge the two groups' (m, l, O) and publish it.
         WARP_WAIT_OR(o_full, pieces & 1, break);
         tc_fence_after();
@@ -1039,8 +1219,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const float M = fmaxf(m_used, o1.x);
           const float a0 = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
           const float a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
-          const long long slot = static_cast<long long>(cur.b) * nseg + cur.seg + blockIdx.x;
-          float* dst = p.part_o + (slot * ROWS + r) * D;
+          const long long pslot = static_cast<long long>(items[slot].z) + blockIdx.x;
+          float* dst = p.part_o + (pslot * ROWS + r) * D;
           if (!idle_warp) {  // rows of all-padding warps are never merged
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
@@ -1062,7 +1242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 *reinterpret_cast<float4*>(dst + c0 + k) = v;
               }
             }
-            p.part_ml[slot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
+            p.part_ml[pslot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
           }
           tc_fence_before();
           __syncwarp();
@@ -1070,9 +1250,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         ++pieces;
       }
-      if (group_last(cur, j, n)) ++gi;
-      cursor_next(cur, p);
+      ++gi;
+      if (flags & kItemEnd) break;
     }
+#undef FAIL
   }
 #undef WAIT_OR
 #undef WARP_WAIT_OR
@@ -1085,14 +1266,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   const int RV = p.Gc * p.K;
-  if (sched[6] >= 0) {
+  const OwnSeg own = read_own();
+  if (own.s >= 0) {
     // Per-segment partition: the cn CTAs of this CTA's segment each add to the
     // segment's counter once their piece is written (the first adds 2^20 -
     // (cn - 1), the rest 1, so every call adds exactly 2^20 and the counter
     // never needs a reset); a CTA's own add pins the call's target.  Then the
     // segment's rows are merged by its own CTAs, an equal share each.
-    const OwnSeg own{sched[6], static_cast<int>(sched[7] >> 32),
-                     static_cast<int>(sched[7] & 0xffffffff), static_cast<int>(sched[8])};
     const int k = static_cast<int>(blockIdx.x) - own.c0;
     const int row0 = static_cast<int>(mul_div(k, RV, own.cn));
     const int row1 = static_cast<int>(mul_div(k + 1, RV, own.cn));
@@ -1155,8 +1335,8 @@ int check_shape(int B, int Hq, int Hkv, int d, int K, Shape* sh) {
 // advances them by fixed amounts, so they never need resetting.
 constexpr size_t WS_TICKET = 256;
 
-size_t counter_bytes(const Shape& sh) {
-  return (static_cast<size_t>(sh.S) * sizeof(unsigned long long) + 255) / 256 * 256;
+size_t counter_bytes(const Shape& sh) {  // completion + claim counters
+  return (2 * static_cast<size_t>(sh.S) * sizeof(unsigned long long) + 255) / 256 * 256;
 }
 
 size_t workspace_bytes(const Shape& sh, int sms) {
@@ -1198,6 +1378,7 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.gbar = reinterpret_cast<unsigned long long*>(w);
   p.seg_cnt = reinterpret_cast<unsigned long long*>(w + WS_TICKET);
+  p.seg_next = p.seg_cnt + sh.S;
   const size_t head = WS_TICKET + counter_bytes(sh);
   p.part_o = reinterpret_cast<float*>(w + head);
   p.part_ml = reinterpret_cast<float2*>(w + head + slots * ROWS * D * sizeof(float));
@@ -1211,7 +1392,8 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   p.Gc = sh.Gc;
   p.nhc = sh.nhc;
   p.cap = cache->cap;
-  p.mask_mode = mask_mode;
+  p.mask_mode = mask_mode & 1;
+  p.balance = (mask_mode & ORTHRUS_ATTN_DETERMINISTIC) ? 0 : 1;
   p.sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
 
   auto* kfn = attn_splitkv_kernel<D>;
@@ -1255,7 +1437,9 @@ extern "C" int orthrus_block_attn(const void* q, const orthrus_kv_cache* cache, 
                                   int mask_mode, void* out, void* workspace, size_t ws_bytes,
                                   int32_t* dev_status, void* stream) {
   if (q == nullptr || cache == nullptr || out == nullptr) return ORTHRUS_EINVAL;
-  if (mask_mode != ORTHRUS_MASK_DIFF && mask_mode != ORTHRUS_MASK_AR) return ORTHRUS_EINVAL;
+  if ((mask_mode & ~ORTHRUS_ATTN_DETERMINISTIC) != ORTHRUS_MASK_DIFF &&
+      (mask_mode & ~ORTHRUS_ATTN_DETERMINISTIC) != ORTHRUS_MASK_AR)
+    return ORTHRUS_EINVAL;
   attn::Shape sh;
   int rc = attn::check_shape(cache->B, Hq, cache->Hkv, cache->d, K, &sh);
   if (rc != ORTHRUS_OK) return rc;

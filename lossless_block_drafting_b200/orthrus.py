@@ -16,6 +16,7 @@ import torch
 
 MASK_DIFF = 0
 MASK_AR = 1
+ATTN_DETERMINISTIC = 0x100  # OR into mask_mode: fixed key ranges, bitwise-repeatable output
 
 OK, EINVAL, ESHAPE, EUNSUPPORTED, ECUDA, ECAPACITY, EWORKSPACE, EALIGN, ETIMEOUT = \
     0, -1, -2, -3, -4, -5, -6, -7, -8

@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 ATOL, RTOL_L2, GAP = 2e-2, 5e-3, 1e-3
 
 
-def attn_gpu(case: synth.AttnCase, mode, dev_status=None):
+def attn_gpu(case: synth.AttnCase, mode, dev_status=None, workspace=None):
     """Run the CUDA path; unless the caller inspects the status itself, assert the
     kernels reported no device-side error (including a bounded wait giving up)."""
     q = case.q.cuda()
@@ -30,7 +30,7 @@ def attn_gpu(case: synth.AttnCase, mode, dev_status=None):
     cl = torch.from_numpy(case.ctx_lens).cuda()
     st = dev_status if dev_status is not None else torch.zeros(1, dtype=torch.int32,
                                                                device="cuda")
-    out = ob.block_attn(q, kc, vc, cl, mode, dev_status=st)
+    out = ob.block_attn(q, kc, vc, cl, mode, dev_status=st, workspace=workspace)
     torch.cuda.synchronize()
     if dev_status is None:
         assert int(st.item()) == 0, ob.status_str(int(st.item()))
@@ -71,12 +71,14 @@ ATTN_CASES = [
 ]
 
 
+@pytest.mark.parametrize("det", [False, True], ids=["balanced", "deterministic"])
 @pytest.mark.parametrize("mode", [ob.MASK_DIFF, ob.MASK_AR])
 @pytest.mark.parametrize("B,K,Hq,Hkv,d,ctx,cap", ATTN_CASES)
-def test_block_attn_matches_oracle(B, K, Hq, Hkv, d, ctx, cap, mode):
+def test_block_attn_matches_oracle(B, K, Hq, Hkv, d, ctx, cap, mode, det):
     case = synth.attn_case(B, K, Hq, Hkv, d, ctx, cap=cap, seed=B * 7 + K + d)
     ref = oracle.block_attn(case.q, case.k_cache, case.v_cache, case.ctx_lens, mode)
-    assert_attn_close(attn_gpu(case, mode), ref)
+    flag = ob.ATTN_DETERMINISTIC if det else 0
+    assert_attn_close(attn_gpu(case, mode | flag), ref)
 
 
 @pytest.mark.parametrize("mode", [ob.MASK_DIFF, ob.MASK_AR])
@@ -135,8 +137,9 @@ def test_block_attn_repeat_calls_same_workspace_are_deterministic():
     q, kc, vc = case.q.cuda(), case.k_cache.cuda(), case.v_cache.cuda()
     cl = torch.from_numpy(case.ctx_lens).cuda()
     ws = torch.zeros(ob.block_attn_workspace_size(2, 32, 8, 128, 32), dtype=torch.uint8, device="cuda")
-    a = ob.block_attn(q, kc, vc, cl, ob.MASK_AR, workspace=ws).clone()
-    b = ob.block_attn(q, kc, vc, cl, ob.MASK_AR, workspace=ws)
+    mode = ob.MASK_AR | ob.ATTN_DETERMINISTIC
+    a = ob.block_attn(q, kc, vc, cl, mode, workspace=ws).clone()
+    b = ob.block_attn(q, kc, vc, cl, mode, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
     # 16 segments (2 sequences x 8 KV heads) <= SMs: each CTA works inside one
@@ -145,6 +148,23 @@ def test_block_attn_repeat_calls_same_workspace_are_deterministic():
     head = ws[:256 + 16 * 8].view(torch.int64).cpu()
     assert int(head[0]) == 0
     assert head[32:48].tolist() == [2 << 20] * 16
+
+
+def test_block_attn_balanced_calls_reuse_the_workspace():
+    """Balanced mode claims key groups from per-segment counters that are
+    rebased on every call: many calls on one workspace, alternating with
+    deterministic calls, all stay within tolerance of the oracle."""
+    case = synth.attn_case(1, 32, 32, 8, 128, [9000], seed=12)
+    ref = oracle.block_attn(case.q, case.k_cache, case.v_cache, case.ctx_lens, ob.MASK_AR)
+    ws = torch.zeros(ob.block_attn_workspace_size(1, 32, 8, 128, 32), dtype=torch.uint8,
+                     device="cuda")
+    for i in range(6):
+        flag = ob.ATTN_DETERMINISTIC if i % 3 == 2 else 0
+        assert_attn_close(attn_gpu(case, ob.MASK_AR | flag, workspace=ws), ref)
+    head = ws[:256 + 16 * 8].view(torch.int64).cpu()
+    assert head[32:40].tolist() == [6 << 20] * 8    # completion counters: 2^20 per call
+    claims = head[40:48].tolist()   # claim counters: rebased by the last balanced call (#4)
+    assert all((c >> 32) == 4 for c in claims), claims
 
 
 def test_block_attn_stream_k_mode_advances_the_grid_ticket():
