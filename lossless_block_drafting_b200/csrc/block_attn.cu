@@ -214,7 +214,94 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane) {
 // Stream-K (S > P): the flat range of T tiles is split evenly.  All counts
 // fit in 32 bits (B * Hkv * cap < 2^31 is checked on the host).
 __device__ void warp_schedule(const Params& p, int P, int c, int lane, bool report_errors,
+                              long long* sched);
+
+// Up to 32 sequences: one load per lane and interleaved scans, no second pass.
+__device__ __forceinline__ void write_sched(long long* sched, int x0, int x1, int TTx, int b,
+                                            int sg, int nb, int L, int s_own, int c0, int cn) {
+  sched[0] = x0;
+  sched[1] = x1;
+  sched[2] = TTx;
+  sched[3] = (static_cast<long long>(b) << 32) | static_cast<unsigned int>(sg);
+  sched[4] = (static_cast<long long>(x0 - TTx - sg * nb) << 32) | static_cast<unsigned int>(L);
+  sched[5] = nb;
+  sched[6] = s_own;
+  sched[7] = (static_cast<long long>(c0) << 32) | static_cast<unsigned int>(cn);
+  sched[8] = (static_cast<long long>(L) << 32) | static_cast<unsigned int>(nb);
+}
+
+__device__ void warp_schedule_small(const Params& p, int P, int c, int lane, bool report_errors,
+                                    long long* sched) {
+  const int nseg = p.Hkv * p.nhc;
+  const int S = p.B * nseg;
+  const bool in = lane < p.B;
+  const int raw = in ? __ldg(p.ctx_lens + lane) : 0;
+  if (report_errors && in && (raw < 0 || raw > p.cap - p.K)) report(p.dev_status, ORTHRUS_ECAPACITY);
+  const int L = in ? clamp_len(raw, p) : 0;
+  const int nb = in ? n_tiles(L, p) : 0;
+  const int u = nseg * nb;
+  const int T = warp_sum(u);
+  const bool segp = S <= P;
+  const int e = (in && segp) ? 1 + static_cast<int>(mul_div(P - S, nb, T)) : 0;
+  const int v = nseg * e;
+  int iv = v, iu = u;  // inclusive scans of v (CTAs) and u (tiles), interleaved
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int yv = __shfl_up_sync(0xFFFFFFFFu, iv, o);
+    const int yu = __shfl_up_sync(0xFFFFFFFFu, iu, o);
+    if (lane >= o) {
+      iv += yv;
+      iu += yu;
+    }
+  }
+  const int rem = P - __shfl_sync(0xFFFFFFFFu, iv, 31);  // < S
+  const int Cx = iv - v, TTx = iu - u;
+  bool found = false;
+  if (in) {
+    if (segp) {
+      const int bs = lane * nseg;
+      const int lo = Cx + min(bs, rem);
+      const int hi = Cx + v + min(bs + nseg, rem);
+      if (c >= lo && c < hi) {
+        found = true;
+        const int rb = max(0, min(nseg, rem - bs));  // segments of b with one more CTA
+        const int local = c - lo;
+        int sg, k, cn;
+        if (local < rb * (e + 1)) {
+          sg = local / (e + 1);
+          k = local - sg * (e + 1);
+          cn = e + 1;
+        } else {
+          const int l2 = local - rb * (e + 1);
+          sg = rb + l2 / e;
+          k = l2 - (sg - rb) * e;
+          cn = e;
+        }
+        const int Ts = TTx + sg * nb;
+        write_sched(sched, Ts + static_cast<int>(mul_div(k, nb, cn)),
+                    Ts + static_cast<int>(mul_div(k + 1, nb, cn)), TTx, lane, sg, nb, L,
+                    bs + sg, c - k, cn);
+      }
+    } else {
+      const int x0s = static_cast<int>(mul_div(c, T, P)), x1s = static_cast<int>(mul_div(c + 1, T, P));
+      if (x1s > x0s && x0s >= TTx && x0s < TTx + u) {
+        found = true;
+        write_sched(sched, x0s, x1s, TTx, lane, (x0s - TTx) / nb, nb, L, -1, 0, 0);
+      }
+    }
+  }
+  if (!__any_sync(0xFFFFFFFFu, found) && lane == 0) {  // no tiles for this CTA
+    for (int i = 0; i < 9; ++i) sched[i] = 0;
+    sched[6] = -1;
+  }
+}
+
+__device__ void warp_schedule(const Params& p, int P, int c, int lane, bool report_errors,
                               long long* sched) {
+  if (p.B <= 32) {
+    warp_schedule_small(p, P, c, lane, report_errors, sched);
+    return;
+  }
   const int nseg = p.Hkv * p.nhc;
   const int S = p.B * nseg;
   int tl = 0;
@@ -473,49 +560,46 @@ __device__ void merge_rows(const Params& p, int P, long long r0, long long r1, i
 }
 
 // Per-segment partition: CTA k of the cn CTAs of segment s merges rows
-// [row0, row1) of that segment, RC rows per round.  One thread bulk-copies the
+// [row0, row1) of that segment, RC rows per round.  Warp 0 bulk-copies the
 // rows' fp32 partial O of up to NPB pieces into shared memory (one contiguous
-// copy per piece, all in flight at once) while every thread loads one (m, l);
-// one warp per row turns the m's into weights against the running row max,
-// then thread (row, float4 column) accumulates the weighted partials and
-// finally writes O / l as bf16.  `buf` is the idle K/V ring (1024-aligned).
+// copy per piece, issued from all lanes, all in flight at once) while other
+// threads load the pieces' (m, l); then thread (row, float4 column) folds the
+// batch into its running (M, L, acc) -- every thread of a row derives the
+// same weights from the shared (m, l) table -- and finally writes acc / L as
+// bf16.  `buf` is the idle K/V ring (1024-aligned).
 template <int D>
 __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int row1, int warp,
                               int lane, uint8_t* buf, volatile int* abort_flag) {
   constexpr int RC = 8;                                  // rows per round
   constexpr int Q4 = D / 4;                              // float4 columns of a row
   constexpr int PIECE = RC * D * 4;                      // bytes of one piece's rows
-  constexpr int HEAD = 8192;                             // barrier, weights, row state
+  constexpr int HEAD = 4096;                             // barrier, (m, l) table
   constexpr int AVAIL = (Layout<D>::NK + Layout<D>::NV) * Layout<D>::KV_BYTES - HEAD;
-  constexpr int NPB = AVAIL / PIECE < THREADS / RC ? AVAIL / PIECE : THREADS / RC;
+  // one (m, l) load per thread of warps 1.., one or two bulk copies per lane of warp 0
+  constexpr int NPB = AVAIL / PIECE < (THREADS - 32) / RC ? AVAIL / PIECE : (THREADS - 32) / RC;
   static_assert(NPB >= 1 && NPB <= 64, "merge batch: 1..64 pieces (two per lane of warp 0)");
+  static_assert(64 + NPB * RC * 8 <= HEAD, "merge (m, l) table");
   const uint32_t bar = smem_u32(buf);
-  float2* ml_s = reinterpret_cast<float2*>(buf + 64);                        // [NPB][RC]
-  float* w_s = reinterpret_cast<float*>(buf + 64 + NPB * RC * 8);             // [NPB][RC]
-  float* row_s = reinterpret_cast<float*>(buf + 64 + NPB * RC * 12);          // M, L, scale
+  float2* ml_s = reinterpret_cast<float2*>(buf + 64);                         // [NPB][RC]
   const float4* o_s = reinterpret_cast<const float4*>(buf + HEAD);            // [NPB][RC][Q4]
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  // every CTA of the segment wrote a piece (or, balanced, an empty one)
-  const bool dense = p.balance || own.cn <= own.ns;
+  const bool dense = p.balance || own.cn <= own.ns;  // every CTA wrote a (maybe empty) piece
   auto live = [&](int j) {
     return dense || mul_div(j, own.ns, own.cn) != mul_div(j + 1, own.ns, own.cn);
   };
   const int nseg = p.Hkv * p.nhc;
   const int b = static_cast<int>(own.s / nseg), seg = static_cast<int>(own.s % nseg);
   const int g = seg / p.nhc, hc = seg % p.nhc;
+  const int tr = threadIdx.x / Q4, tq = threadIdx.x % Q4;  // this thread's (row, float4)
   uint32_t phase = 0;
   for (int rb = row0; rb < row1; rb += RC) {
     const int nr = row1 - rb < RC ? row1 - rb : RC;
-    if (threadIdx.x < RC) {
-      row_s[threadIdx.x] = -INFINITY;       // running max
-      row_s[RC + threadIdx.x] = 0.f;        // running normaliser
-    }
-    const int tr = threadIdx.x / Q4, tq = threadIdx.x % Q4;  // this thread's (row, float4)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float M = -INFINITY, L = 0.f;
     for (int j0 = 0; j0 < own.cn; j0 += NPB) {
       const int nb = own.cn - j0 < NPB ? own.cn - j0 : NPB;
       if (warp == 0) {
@@ -536,56 +620,38 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
           bulk_load(smem_u32(buf + HEAD + jj * PIECE), p.part_o + (slot * ROWS + rb) * D,
                     nr * D * 4, bar);
         }
-      }
-      if (threadIdx.x < nb * RC) {
-        const int jj = threadIdx.x / RC, r = threadIdx.x % RC;
+      } else if (threadIdx.x - 32 < nb * RC) {
+        const int t = threadIdx.x - 32;
+        const int jj = t / RC, r = t % RC;
         const long long slot = own.s + own.c0 + j0 + jj;
-        ml_s[threadIdx.x] = (r < nr && live(j0 + jj)) ? __ldcg(p.part_ml + slot * ROWS + rb + r)
-                                                      : make_float2(-INFINITY, 0.f);
-      }
-      __syncthreads();
-      if (warp < nr) {
-        // Row `warp`: batch max, weights, running (M, L) and the rescale of acc.
-        const int r = warp;
-        float mb = -INFINITY;
-        for (int jj = lane; jj < nb; jj += 32) mb = fmaxf(mb, ml_s[jj * RC + r].x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
-        const float m_old = row_s[r];
-        const float m_new = fmaxf(m_old, mb);
-        float lb = 0.f;
-        for (int jj = lane; jj < nb; jj += 32) {
-          const float2 ml = ml_s[jj * RC + r];
-          const float wj = ml.x == -INFINITY ? 0.f : fast_exp2(ml.x - m_new);
-          w_s[jj * RC + r] = wj;
-          lb += wj * ml.y;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) lb += __shfl_xor_sync(0xFFFFFFFFu, lb, o);
-        if (lane == 0) {
-          const float sc = m_old == -INFINITY ? 0.f : fast_exp2(m_old - m_new);
-          row_s[r] = m_new;
-          row_s[RC + r] = row_s[RC + r] * sc + lb;
-          row_s[2 * RC + r] = sc;
-        }
+        ml_s[t] = (r < nr && live(j0 + jj)) ? __ldcg(p.part_ml + slot * ROWS + rb + r)
+                                            : make_float2(-INFINITY, 0.f);
       }
       mbar_wait_bounded(bar, phase, abort_flag, p.dev_status);  // gives up: status set
       phase ^= 1u;
       __syncthreads();
       if (tr < nr) {
-        const float sc = row_s[2 * RC + tr];
-        acc.x *= sc;
-        acc.y *= sc;
-        acc.z *= sc;
-        acc.w *= sc;
-        for (int jj = 0; jj < nb; ++jj) {
-          const float wj = w_s[jj * RC + tr];
-          if (wj == 0.f) continue;  // dead piece or no mass: its rows may be stale
-          const float4 x = o_s[(jj * RC + tr) * Q4 + tq];
-          acc.x += wj * x.x;
-          acc.y += wj * x.y;
-          acc.z += wj * x.z;
-          acc.w += wj * x.w;
+        float mb = M;
+        for (int jj = 0; jj < nb; ++jj) mb = fmaxf(mb, ml_s[jj * RC + tr].x);
+        if (mb != -INFINITY) {
+          const float sc = M == -INFINITY ? 0.f : fast_exp2(M - mb);
+          acc.x *= sc;
+          acc.y *= sc;
+          acc.z *= sc;
+          acc.w *= sc;
+          L *= sc;
+          M = mb;
+          for (int jj = 0; jj < nb; ++jj) {
+            const float2 ml = ml_s[jj * RC + tr];
+            if (ml.x == -INFINITY) continue;  // dead or empty piece: its O may be stale
+            const float wj = fast_exp2(ml.x - M);
+            const float4 x = o_s[(jj * RC + tr) * Q4 + tq];
+            L += wj * ml.y;
+            acc.x += wj * x.x;
+            acc.y += wj * x.y;
+            acc.z += wj * x.z;
+            acc.w += wj * x.w;
+          }
         }
       }
       __syncthreads();
@@ -594,7 +660,6 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
       const int row = rb + tr;
       const int i = row / p.Gc, hh = row % p.Gc;
       if (hc * p.Gc + hh < p.G) {
-        const float L = row_s[RC + tr];
         const float inv = L > 0.f ? 1.f / L : 0.f;
         const int h = g * p.G + hc * p.Gc + hh;
         __nv_bfloat16* dst =
@@ -605,7 +670,6 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
         *reinterpret_cast<uint2*>(dst) = pk;
       }
     }
-    __syncthreads();
   }
 }
 
@@ -687,27 +751,33 @@ __global__ void __launch_bounds__(THREADS, 1)
   OwnSeg pr_own{-1, 0, 0, 0, 0};
   Cursor pr_c{};
   int pr_n = 0, pr_j = 0, pr_cur = -2;
-  int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0, pr_have = 0, pr_bnext = 0;
+  int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0;
   bool pr_grabbing = false, pr_dry = true;
   unsigned long long pr_base = 0, pr_pend = 0;
   const uint64_t pr_policy = policy_evict_first();
-  auto emit = [&](int t, int L, long long s, int flags) -> bool {
+  int pr_s = -1, pr_kvbase = 0, pr_qh = 0, pr_qb = 0;  // cached for the current segment
+  auto emit = [&](int t, int L, int s, int flags) -> bool {
     const int slot = pr_gi % RING;
-    const int b = static_cast<int>(s / nseg), seg = static_cast<int>(s % nseg);
-    const int g = seg / p.nhc, hc = seg % p.nhc;
-    const int kvbase = (b * p.Hkv + g) * p.cap;
+    if (s != pr_s && s >= 0) {
+      pr_s = s;
+      const int b = s / nseg, seg = s - b * nseg;
+      const int g = seg / p.nhc, hc = seg - g * p.nhc;
+      pr_kvbase = (b * p.Hkv + g) * p.cap;
+      pr_qh = g * p.G + hc * p.Gc;
+      pr_qb = b * p.K;
+    }
+    const int kvbase = pr_kvbase;
     // Ring slots are never overwritten early: the producer is at most NK
     // groups ahead of S = Q K^T, which is at most NSB groups ahead of P V,
     // which trails every other reader of an item (RING > NK + NSB + 1).
-    items[slot] = make_int4(t | (flags << kItemFlagShift), L, static_cast<int>(s), kvbase);
+    items[slot] = make_int4(t | (flags << kItemFlagShift), L, s, kvbase);
     mbar_arrive(item_full(slot));
     if (flags & kItemNone) return true;
     if (flags & kItemPieceFirst) {
       if (!mbar_wait_bounded(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status)) return false;
       mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.Gc * p.K * D * 2));
       for (int c = 0; c < Ly::CHUNKS; ++c)
-        tma_load_3d(sb0 + Ly::OFF_Q + c * Ly::Q_CHUNK, &tmQ, q_full, c * 64,
-                    g * p.G + hc * p.Gc, b * p.K);
+        tma_load_3d(sb0 + Ly::OFF_Q + c * Ly::Q_CHUNK, &tmQ, q_full, c * 64, pr_qh, pr_qb);
       ++pr_pieces;
     }
     const bool pair = flags & kItemPair;
@@ -723,8 +793,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   };
   // Balanced per-segment partition: the CTA first streams a static run of
   // about 3/4 of its fair share of the segment's 128-key groups, then claims
-  // groups of the remaining pool two at a time from the segment's claim
-  // counter (one claim kept in flight, so its latency is hidden).  The
+  // groups of the remaining pool one at a time from the segment's claim
+  // counter (the next claim is always in flight, so its latency is hidden,
+  // and siblings finish within about one group of each other).  The
   // counter is rebased per call to epoch E << 32, E being the number of
   // completed calls read from the segment's completion counter (which cannot
   // reach the next multiple of 2^20 before this CTA's own add).
@@ -733,7 +804,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         *reinterpret_cast<volatile unsigned long long*>(p.seg_cnt + pr_own.s);
     pr_base = (done >> 20) << 32;
     atomicMax(p.seg_next + pr_own.s, pr_base);
-    pr_pend = atomicAdd(p.seg_next + pr_own.s, 2ull);
+    pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);
     pr_grabbing = true;
   };
   auto next_group = [&]() -> int {
@@ -744,22 +815,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (pr_dry) return -1;
     if (!pr_grabbing) start_claims();
-    if (pr_have == 0) {
-      const long long first = pr_pool0 + static_cast<long long>(pr_pend - pr_base);
-      if (first >= pr_ngr) {
-        pr_dry = true;
-        return -1;
-      }
-      pr_bnext = static_cast<int>(first);
-      pr_have = 2;
-      pr_pend = atomicAdd(p.seg_next + pr_own.s, 2ull);  // next claim, in flight
-    }
-    --pr_have;
-    if (pr_bnext >= pr_ngr) {
+    const long long g = pr_pool0 + static_cast<long long>(pr_pend - pr_base);
+    if (g >= pr_ngr) {
       pr_dry = true;
       return -1;
     }
-    return pr_bnext++;
+    pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);  // next claim, in flight
+    return static_cast<int>(g);
   };
   // Before the barrier (pre) no other role runs yet, so only groups that need
   // no wait are emitted: the first NK (fresh K stages) of the first piece.
@@ -767,14 +829,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (pr_own.s >= 0 && p.balance) {
       if (pr_cur == -2) {
         pr_cur = next_group();
-        if (pr_cur < 0) emit(0, pr_own.L, pr_own.s, kItemNone);
+        if (pr_cur < 0) emit(0, pr_own.L, static_cast<int>(pr_own.s), kItemNone);
       }
       while (pr_cur >= 0 && pr_gi < limit) {
         const int nxt = next_group();
         const bool pair = 2 * pr_cur + 1 < pr_own.ns;
         const int flags = (pair ? kItemPair : 0) | (pr_gi == 0 ? kItemPieceFirst : 0) |
                           (nxt < 0 ? (kItemPieceLast | kItemEnd) : 0);
-        if (!emit(2 * pr_cur, pr_own.L, pr_own.s, flags)) {
+        if (!emit(2 * pr_cur, pr_own.L, static_cast<int>(pr_own.s), flags)) {
           pr_cur = -1;
           break;
         }
@@ -784,7 +846,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // Static range [x0, x0 + n) of the flat tile space (deterministic).
       if (pr_cur == -2) {
         pr_cur = 0;
-        if (pr_n == 0) emit(0, 0, pr_own.s, kItemNone);
+        if (pr_n == 0) emit(0, 0, static_cast<int>(pr_own.s), kItemNone);
       }
       while (pr_j < pr_n && pr_gi < limit) {
         const bool pair = !group_last(pr_c, pr_j, pr_n);
@@ -794,7 +856,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int flags = (pair ? kItemPair : 0) | (pfirst ? kItemPieceFirst : 0) |
                           (plast ? kItemPieceLast : 0) | (jl == pr_n - 1 ? kItemEnd : 0);
         if (pre && pfirst && pr_pieces > 0) break;  // its Q waits for the previous piece's
-        if (!emit(pr_c.t, pr_c.L, static_cast<long long>(pr_c.b) * nseg + pr_c.seg, flags)) {
+        if (!emit(pr_c.t, pr_c.L, pr_c.b * nseg + pr_c.seg, flags)) {
           pr_j = pr_n;
           break;
         }
@@ -823,7 +885,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(p_full(2 * i + 1), 4);
     }
     mbar_init(o_full, 1);
-    mbar_init(o_free, 4);
+    mbar_init(o_free, 8);
     mbar_init(mma_done, 2);
     for (int i = 0; i < RING; ++i) mbar_init(item_full(i), 1);
     *abort_flag = 0;
@@ -1090,78 +1152,34 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int tile0 = (t0 + h) * TN;
         WARP_WAIT_OR(s_full(gb), (gi >> 1) & 1, FAIL);
         tc_fence_after();
-        uint32_t sr[TN];
-        tmem_ld64(t_s, sr);
-        tmem_wait_ld();
-
-        if (tile0 + TN > Lc + 1) {
-          // Tail tile: some keys lie past some row's limit.  Interior tiles
-          // (every key < L + 1) skip this entirely.
-          const int lim = (r >= rows_valid) ? 0
-                          : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : Lc + i_row + 1);
-#pragma unroll
-          for (int c = 0; c < TN; ++c)
-            if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-        }
         // p = 2^(s*sl2 - m) against the running reference m (scale and shift as
-        // packed f32x2 FMAs, exp2 on the SFU, row sum as packed adds); the
-        // tile max is computed alongside and only a jump of the max by more
-        // than 2^8 forces the slow path that rescales O and redoes the tile.
-        // The first tile of a piece takes its own max first.
+        // packed f32x2 FMAs, exp2 on the SFU, row sum as packed adds).  Pass 0
+        // is the common case; the first tile of a piece takes its own max
+        // first.  Every p is positive, so a tile row sum of at most 2^8 proves
+        // no element exceeded the reference by more than 2^8: only otherwise
+        // (rare) does pass 1 reload S, take the tile max, rescale O_w and l
+        // and redo the tile.  One copy of the tile code keeps the hot loop
+        // small in the instruction cache.
         const float2 sc2 = make_float2(sl2, sl2);
         float x[TN];
         float2 acc2[4];
-        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        // exps against m_ref, also folding the tile max when want_max (each S
-        // value is read once, so S and P are never both live in registers)
-        auto exps = [&](float m_ref, bool want_max) {
-          const float m_eff = (m_ref == -INFINITY) ? 0.f : m_ref;
-          const float2 nm2 = make_float2(-m_eff, -m_eff);
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+          uint32_t sr[TN];
+          tmem_ld64(t_s, sr);
+          tmem_wait_ld();
+          if (tile0 + TN > Lc + 1) {
+            // Tail tile: some keys lie past some row's limit.  Interior tiles
+            // (every key < L + 1) skip this entirely.
+            const int lim = (r >= rows_valid) ? 0
+                            : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : Lc + i_row + 1);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc2[q] = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int c = 0; c < TN; c += 2) {
-            const float s0 = __uint_as_float(sr[c]), s1 = __uint_as_float(sr[c + 1]);
-            if (want_max) mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], s0, s1);
-            const float2 a2 = __ffma2_rn(make_float2(s0, s1), sc2, nm2);
-            const float2 e2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-            x[c] = e2.x;
-            x[c + 1] = e2.y;
-            acc2[(c >> 1) & 3] = __fadd2_rn(acc2[(c >> 1) & 3], e2);
+            for (int c = 0; c < TN; ++c)
+              if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
           }
-        };
-        auto reduce_max = [&]() {
-          return fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
-        };
-        if (fresh) {
-#pragma unroll
-          for (int c = 0; c < TN; c += 8) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
-                             __uint_as_float(sr[c + 2 * q + 1]));
-          }
-          m_used = reduce_max();
-          exps(m_used, false);
-        } else {
-          // Every p is positive, so a tile row sum of at most 2^8 proves no
-          // element exceeded the reference by more than 2^8: the sums the row
-          // needs anyway decide whether the (rare) rescale path runs, and only
-          // then is the tile max taken.
-          exps(m_used, false);
-          const float2 ts2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
-          if (__any_sync(0xFFFFFFFFu, !(ts2.x + ts2.y <= 256.f))) {
-            // S is still in its TMEM buffer: reload it (re-masked), take the
-            // tile max, rescale O_w and l, and redo the tile.
-            tmem_ld64(t_s, sr);
-            tmem_wait_ld();
-            if (tile0 + TN > Lc + 1) {
-              const int lim = (r >= rows_valid) ? 0
-                              : (p.mask_mode == ORTHRUS_MASK_DIFF ? kv_end : Lc + i_row + 1);
-#pragma unroll
-              for (int c = 0; c < TN; ++c)
-                if (tile0 + c >= lim) sr[c] = __float_as_uint(-INFINITY);
-            }
+          const bool take_max = fresh || pass == 1;
+          if (take_max) {
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < TN; c += 8) {
 #pragma unroll
@@ -1169,29 +1187,50 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mx4[q] = fmax3(mx4[q], __uint_as_float(sr[c + 2 * q]),
                                __uint_as_float(sr[c + 2 * q + 1]));
             }
-            const float mx = reduce_max();
-            const float m_new = fmaxf(m_used, mx);
-            const float f = (m_new == -INFINITY) ? 1.f
-                            : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
-            // O_w may only be touched once this group's previous P*V (tile
-            // j - 2, in load group prev_gi) has completed.
-            WARP_WAIT_OR(sb_free(prev_gi & 1), (prev_gi >> 1) & 1, FAIL);
-            tc_fence_after();
+            const float mx = fmax3(fmaxf(mx4[0], mx4[1]), mx4[2], mx4[3]) * sl2;
+            if (pass == 0) {
+              m_used = mx;
+            } else {
+              const float m_new = fmaxf(m_used, mx);
+              const float f = (m_new == -INFINITY) ? 1.f
+                              : (m_used == -INFINITY ? 0.f : fast_exp2(m_used - m_new));
+              // O_w may only be touched once this group's previous P*V (tile
+              // j - 2, in load group prev_gi) has completed.
+              WARP_WAIT_OR(sb_free(prev_gi & 1), (prev_gi >> 1) & 1, FAIL);
+              tc_fence_after();
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(t_o + c0, o);
-              tmem_wait_ld();
+              for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t o[16];
+                tmem_ld16(t_o + c0, o);
+                tmem_wait_ld();
 #pragma unroll
-              for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
-              tmem_st16(t_o + c0, o);
+                for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * f);
+                tmem_st16(t_o + c0, o);
+              }
+              tmem_wait_st();
+              l_sum *= f;
+              m_used = m_new;
             }
-            tmem_wait_st();
-            l_sum *= f;
-            m_used = m_new;
-            exps(m_used, false);
           }
+          // each S value is read once, so S and P are never both live in registers
+          const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+          const float2 nm2 = make_float2(-m_eff, -m_eff);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc2[q] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < TN; c += 2) {
+            const float2 a2 = __ffma2_rn(
+                make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
+            const float2 e2 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+            x[c] = e2.x;
+            x[c + 1] = e2.y;
+            acc2[(c >> 1) & 3] = __fadd2_rn(acc2[(c >> 1) & 3], e2);
+          }
+          if (take_max) break;
+          const float2 ts2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
+          if (!__any_sync(0xFFFFFFFFu, !(ts2.x + ts2.y <= 256.f))) break;
         }
+        if (fail) break;
         const float2 t2 = __fadd2_rn(__fadd2_rn(acc2[0], acc2[1]), __fadd2_rn(acc2[2], acc2[3]));
         l_sum += t2.x + t2.y;
 
@@ -1209,45 +1248,56 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (fail) break;
 
       if (flags & kItemPieceLast) {
-        // Piece epilogue: merge the two groups' (m, l, O) and publish it.
+        // Piece epilogue: merge the two groups' (m, l, O) and publish it.  WG1
+        // hands its (m, l) to WG0, which writes the row's (M, l) and hands
+        // back the two scales; then each group writes half of the columns.
         WARP_WAIT_OR(o_full, pieces & 1, break);
         tc_fence_after();
+        const long long pslot = static_cast<long long>(items[slot].z) + blockIdx.x;
         if (w == 1) ml_xchg[r] = make_float2(m_used, l_sum);
         asm volatile("bar.sync 1, 256;" ::: "memory");
+        float a0, a1;
         if (w == 0) {
           const float2 o1 = ml_xchg[r];
           const float M = fmaxf(m_used, o1.x);
-          const float a0 = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
-          const float a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
-          const long long pslot = static_cast<long long>(items[slot].z) + blockIdx.x;
-          float* dst = p.part_o + (pslot * ROWS + r) * D;
-          if (!idle_warp) {  // rows of all-padding warps are never merged
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t o0[32], o1r[32];
-              tmem_ld32(t_o + c0, o0);
-              tmem_ld32(t_o + 128 + c0, o1r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int k = 0; k < 32; k += 4) {
-                float4 v;
-                v.x = (a0 != 0.f ? a0 * __uint_as_float(o0[k]) : 0.f) +
-                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k]) : 0.f);
-                v.y = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 1]) : 0.f) +
-                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 1]) : 0.f);
-                v.z = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 2]) : 0.f) +
-                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
-                v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
-                      (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
-                *reinterpret_cast<float4*>(dst + c0 + k) = v;
-              }
-            }
-            p.part_ml[pslot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
+          a0 = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
+          a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
+          if (!idle_warp) p.part_ml[pslot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
         }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (w == 0) ml_xchg[r] = make_float2(a0, a1);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (w == 1) {
+          const float2 sc = ml_xchg[r];
+          a0 = sc.x;
+          a1 = sc.y;
+        }
+        if (!idle_warp) {  // rows of all-padding warps are never merged
+          float* dst = p.part_o + (pslot * ROWS + r) * D;
+#pragma unroll
+          for (int c0 = w * (D / 2); c0 < (w + 1) * (D / 2); c0 += 32) {
+            uint32_t o0[32], o1r[32];
+            tmem_ld32(lane_base + TMEM_O + c0, o0);
+            tmem_ld32(lane_base + TMEM_O + 128 + c0, o1r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; k += 4) {
+              float4 v;
+              v.x = (a0 != 0.f ? a0 * __uint_as_float(o0[k]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k]) : 0.f);
+              v.y = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 1]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 1]) : 0.f);
+              v.z = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 2]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
+              v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
+                    (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
+              *reinterpret_cast<float4*>(dst + c0 + k) = v;
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free);  // all 8 softmax warps are done with O
         ++pieces;
       }
       ++gi;

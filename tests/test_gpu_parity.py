@@ -68,6 +68,8 @@ ATTN_CASES = [
     (1, 32, 8, 2, 128, [6000], None),              # 2 segments x 74 CTAs: merge in 2 batches
     (1, 32, 12, 2, 64, [500], None),               # G = 6 over 4-head chunks: padding heads
     (20, 4, 16, 8, 64, list(range(60, 1260, 60)), None),  # 160 segments > 148 CTAs
+    (36, 4, 2, 1, 64, [17 * i % 300 for i in range(36)], None),  # B > 32, 36 segments
+    (40, 2, 8, 4, 64, [5 + 29 * i % 700 for i in range(40)], None),  # B > 32, stream-K
 ]
 
 
