@@ -225,13 +225,26 @@ class Workload:
 
         self.k = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
         self.v = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
-        self.q_diff = [randn(B, K, Hq, d) for _ in range(layers)]
-        self.q_ar = [randn(B, K, Hq, d) for _ in range(layers)]
+        # A step's inputs (both views' queries for every layer, both views' final
+        # hidden states) live in one flat buffer, so one host->device copy
+        # delivers them all in the end-to-end measurement.
+        n_q, n_h = B * K * Hq * d, B * K * H
+        self.inputs = torch.empty(2 * layers * n_q + 2 * n_h, dtype=bf, device=device)
+        off = [0]
+
+        def place(x):
+            v = self.inputs[off[0]:off[0] + x.numel()].view(x.shape)
+            v.copy_(x)
+            off[0] += x.numel()
+            return v
+
+        self.q_diff = [place(randn(B, K, Hq, d)) for _ in range(layers)]
+        self.q_ar = [place(randn(B, K, Hq, d)) for _ in range(layers)]
         self.W = randn(V, H, std=0.02)
-        self.h_ar = randn(B * K, H)
+        self.h_ar = place(randn(B * K, H))
         # the diffusion view's final states agree with the AR view's on the first
         # `accept` rows of every block, so drafts match the AR argmax there
-        self.h_diff = randn(B * K, H)
+        self.h_diff = place(randn(B * K, H))
         a = max(0, min(accept, K))
         hv = self.h_diff.view(B, K, H)
         hv[:, :a] = self.h_ar.view(B, K, H)[:, :a]
@@ -463,12 +476,9 @@ def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):
     """Same metric end to end: per step, H2D of the step's inputs from pinned host
     memory, the captured step (public C-ABI calls), and a D2H read of the results."""
     import torch
-    host_in = []
-    for i in range(wl.layers):
-        host_in.append((wl.q_diff[i].cpu().pin_memory(), wl.q_diff[i]))
-        host_in.append((wl.q_ar[i].cpu().pin_memory(), wl.q_ar[i]))
-    host_in.append((wl.h_diff.cpu().pin_memory(), wl.h_diff))
-    host_in.append((wl.h_ar.cpu().pin_memory(), wl.h_ar))
+    # every input of the step (queries of both views for all layers, both views'
+    # hidden states) in one pinned buffer -> one copy into the flat device buffer
+    host_in = [(wl.inputs.cpu().pin_memory(), wl.inputs)]
     outs = [wl.accept_len, wl.next_tok, wl.ctx_lens]
     host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
     h2d = sum(h.numel() * h.element_size() for h, _ in host_in)
