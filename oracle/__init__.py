@@ -62,9 +62,12 @@ def _load():
             lib.oracle_row_argmax.argtypes = [P, I, I, I, P, P, P]
             lib.oracle_verify.argtypes = [P, P, I, I, P, P]
             lib.oracle_kv_commit.argtypes = [P, P, I, I, I, P]
+            D = ctypes.c_double
+            lib.oracle_qkv_append.argtypes = [P, I, P, P, I, D, D, P, I, I, I, I, I, I,
+                                              P, P, P]
             for f in ("oracle_block_attn", "oracle_lmhead_argmax", "oracle_row_argmax",
                       "oracle_verify", "oracle_kv_commit", "oracle_version",
-                      "oracle_num_threads"):
+                      "oracle_num_threads", "oracle_qkv_append"):
                 getattr(lib, f).restype = I
             _lib = lib
     return _lib
@@ -210,3 +213,42 @@ def kv_commit(ctx_lens, accept_len, K: int, cap: int):
     if rc != OK:
         raise ValueError(f"oracle_kv_commit failed with status {rc}")
     return cl, int(st[0])
+
+
+def qkv_append(qkv, ctx_lens, K: int, Hq: int, Hkv: int, d: int, k_cache, v_cache,
+               q_norm_w=None, k_norm_w=None, theta: float = 1e6, eps: float = 1e-6):
+    """Block Q/K/V append: per-head RMS norm of q and k (if weights are given),
+    rotary embedding at positions L_b + i, K/V written into slots [L_b, L_b + K).
+
+    qkv [B*K, (Hq + 2 Hkv) d] (token-major, heads packed q | k | v); ctx_lens [B];
+    k_cache, v_cache fp64 [B, Hkv, cap, d], updated in place (a copy is made if
+    they are not writable fp64 arrays, and the updated arrays are returned).
+    Returns (q_out fp64 [B, K, Hq, d], k_cache, v_cache).
+    """
+    lib = _load()
+    xa, xdt = _as_float_input(qkv)
+    cl = _as_i32(ctx_lens)
+    B = cl.shape[0]
+    if xa.shape != (B * K, (Hq + 2 * Hkv) * d):
+        raise ValueError("qkv shape mismatch")
+    kc = np.ascontiguousarray(np.asarray(k_cache, dtype=np.float64)).copy()
+    vc = np.ascontiguousarray(np.asarray(v_cache, dtype=np.float64)).copy()
+    if kc.shape != vc.shape or kc.shape[:2] != (B, Hkv) or kc.shape[3] != d:
+        raise ValueError("cache shape mismatch")
+    cap = kc.shape[2]
+    qw = kw = None
+    wdt = F64
+    if q_norm_w is not None or k_norm_w is not None:
+        if q_norm_w is None or k_norm_w is None:
+            raise ValueError("give both norm weights or neither")
+        qw, wdt = _as_float_input(q_norm_w)
+        kw, wdt2 = _as_float_input(k_norm_w)
+        if wdt2 != wdt:
+            raise TypeError("norm weights must share a dtype")
+    q_out = np.empty((B, K, Hq, d), np.float64)
+    rc = lib.oracle_qkv_append(_ptr(xa), xdt, _ptr(qw), _ptr(kw), wdt, float(theta),
+                               float(eps), _ptr(cl), B, K, Hq, Hkv, d, cap, _ptr(q_out),
+                               _ptr(kc), _ptr(vc))
+    if rc != OK:
+        raise ValueError(f"oracle_qkv_append failed with status {rc}")
+    return q_out, kc, vc

@@ -281,3 +281,88 @@ int oracle_kv_commit(int32_t *ctx_lens, const int32_t *accept_len, int B, int K,
   if (status) *status = st;
   return ORC_OK;
 }
+
+/*
+ * Block Q/K/V append: the step just before block attention, which writes the
+ * block's keys and values into the scratch slots [L_b, L_b + K) of the shared
+ * cache ([GIST 2.1, 2.3 item 1]: the block's K/V live in the one cache;
+ * [ABS]: O(1) overhead).  The pages do not describe the projections' epilogue;
+ * this follows the plain definitions of the Qwen3 family the build targets
+ * (per-head RMS normalisation of q and k, then rotary position embedding):
+ *
+ * Token i of sequence b sits at position p = L_b + i.  qkv is packed per token
+ * as [Hq heads of q | Hkv heads of k | Hkv heads of v], each head d values.
+ *   norm (q and k heads, only if the weight pointer is non-NULL):
+ *     x_c <- x_c / sqrt((1/d) sum_c x_c^2 + eps) * w_c
+ *   rotary embedding, coordinate j paired with j + d/2 (j < d/2):
+ *     a_j = p * theta^(-2j/d)                   (exactly, in fp64)
+ *     y_j       = x_j cos a_j - x_{j+d/2} sin a_j
+ *     y_{j+d/2} = x_{j+d/2} cos a_j + x_j sin a_j
+ *   q_out[b, i, h, :] = rotary(norm_q(q));   k_cache[b, g, p, :] = rotary(norm_k(k));
+ *   v_cache[b, g, p, :] = v.
+ * The caches are fp64 [B, Hkv, cap, d] and only slots [L_b, L_b + K) are
+ * written.  Returns ORC_ECAPACITY (writing nothing) if some L_b + K > cap.
+ */
+int oracle_qkv_append(const void *qkv, int qkv_dtype, const void *q_w, const void *k_w,
+                      int w_dtype, double theta, double eps, const int32_t *ctx_lens, int B,
+                      int K, int Hq, int Hkv, int d, int cap, double *q_out, double *k_cache,
+                      double *v_cache) {
+  if (B < 0 || K < 1 || Hq < 1 || Hkv < 1 || d < 2 || d % 2 || cap < 0 || theta <= 0 ||
+      eps < 0)
+    return ORC_EINVAL;
+  if (Hq % Hkv != 0) return ORC_EINVAL;
+  for (int b = 0; b < B; ++b)
+    if (ctx_lens[b] < 0 || (long)ctx_lens[b] + K > cap) return ORC_ECAPACITY;
+  const int G = Hq / Hkv;
+  const int W = Hq + 2 * Hkv; /* heads per token in qkv */
+  const long ntok = (long)B * K;
+  int err = ORC_OK;
+
+#pragma omp parallel for schedule(static)
+  for (long t = 0; t < ntok; ++t) {
+    const int b = (int)(t / K), i = (int)(t % K);
+    const long pos = (long)ctx_lens[b] + i;
+    double *x = (double *)malloc(sizeof(double) * (size_t)d);
+    double *y = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!x || !y) {
+      free(x);
+      free(y);
+#pragma omp atomic write
+      err = ORC_ENOMEM;
+      continue;
+    }
+    for (int hh = 0; hh < W; ++hh) {
+      const int is_q = hh < Hq, is_k = !is_q && hh < Hq + Hkv;
+      for (int c = 0; c < d; ++c) x[c] = rd(qkv, ((size_t)t * W + hh) * d + c, qkv_dtype);
+      if (is_q || is_k) {
+        const void *w = is_q ? q_w : k_w;
+        if (w) {
+          double ss = 0.0;
+          for (int c = 0; c < d; ++c) ss += x[c] * x[c];
+          const double r = 1.0 / sqrt(ss / d + eps);
+          for (int c = 0; c < d; ++c) x[c] = x[c] * r * rd(w, (size_t)c, w_dtype);
+        }
+        for (int j = 0; j < d / 2; ++j) {
+          const double a = (double)pos * pow(theta, -2.0 * j / d);
+          const double cs = cos(a), sn = sin(a);
+          y[j] = x[j] * cs - x[j + d / 2] * sn;
+          y[j + d / 2] = x[j + d / 2] * cs + x[j] * sn;
+        }
+      } else {
+        for (int c = 0; c < d; ++c) y[c] = x[c];
+      }
+      if (is_q) {
+        double *o = q_out + (((size_t)b * K + i) * Hq + hh) * d;
+        for (int c = 0; c < d; ++c) o[c] = y[c];
+      } else {
+        const int g = is_k ? hh - Hq : hh - Hq - Hkv;
+        double *dst = (is_k ? k_cache : v_cache) + (((size_t)b * Hkv + g) * cap + pos) * d;
+        for (int c = 0; c < d; ++c) dst[c] = y[c];
+      }
+    }
+    free(x);
+    free(y);
+  }
+  (void)G;
+  return err;
+}
