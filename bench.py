@@ -403,6 +403,10 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(wl, g_warm, stream, K_steps, W_steps, world, dev)
+    try:  # an auxiliary measurement: its failure is reported, not fatal to the step's line
+        qkv_append = time_qkv_append(wl, stream)
+    except Exception as exc:  # noqa: BLE001
+        qkv_append = {"error": f"{type(exc).__name__}: {exc}"}
 
     del g_timed, g_warm
     result = {
@@ -456,6 +460,7 @@ def run_ours(args):
             "traffic": measured_traffic(wl),
             "algorithmic_bytes_per_launch": wl.attn_bytes(),
         },
+        "qkv_append": qkv_append,
         "gpu_launches": wl.launches_per_step * K_steps,
         "device_status": status,
         "clocks": clocks,
@@ -470,6 +475,49 @@ def run_ours(args):
         sync_ranks()
         dist.destroy_process_group()
     return result if rank == 0 else None
+
+
+def time_qkv_append(wl: "Workload", stream, launches: int = 100):
+    """The block Q/K/V append (per-head RMS norm, rotary embedding, block K/V into
+    the cache) for one layer at this workload's shapes: device time per launch
+    from a CUDA graph of back-to-back launches.  Reported beside the step, not
+    inside it (the step is the path from the block's queries onwards)."""
+    import torch
+    from lossless_block_drafting_b200 import orthrus as ob
+    Hq, Hkv, d = QWEN["Hq"], QWEN["Hkv"], QWEN["d"]
+    g = torch.Generator(device=wl.k[0].device).manual_seed(99)
+    qkv = torch.randn(wl.B * wl.K, (Hq + 2 * Hkv) * d, generator=g, device=wl.k[0].device,
+                      dtype=torch.float32).to(torch.bfloat16)
+    w = (1 + 0.1 * torch.randn(2, d, generator=g, device=wl.k[0].device)).to(torch.bfloat16)
+    ctx = wl.ctx_init.clone()
+    view = ob.kv_cache_view(wl.k[0], wl.v[0], ctx)
+    q_out = torch.empty(wl.B, wl.K, Hq, d, dtype=torch.bfloat16, device=qkv.device)
+
+    def one():
+        ob.block_qkv_append(qkv, None, None, None, Hq, wl.K, q_norm_w=w[0], k_norm_w=w[1],
+                            q_out=q_out, cache_view=view, stream=stream, dev_status=wl.status)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for _ in range(launches):
+                one()
+        graph.replay()
+        stream.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        graph.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / launches
+    nbytes = 2 * (2 * wl.B * wl.K * (Hq + 2 * Hkv) * d + 2 * d)  # read qkv + weights, write q/k/v
+    del graph
+    return {"us_per_call": round(us, 2), "bytes_per_call": nbytes,
+            "GB_per_s": round(nbytes / (us * 1e-6) / 1e9, 1),
+            "bound": "launch latency (0.8 MB per call)", "in_step": False}
 
 
 def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):

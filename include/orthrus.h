@@ -242,6 +242,37 @@ int orthrus_verify_commit(const int32_t *argmax, const int32_t *draft, int B, in
                           int32_t *accept_len, int32_t *next_tok,
                           const orthrus_kv_cache *cache, int32_t *dev_status, void *stream);
 
+/*
+ * Block Q/K/V append: the step just before orthrus_block_attn, writing the
+ * block's keys and values into the scratch slots [L_b, L_b + K) of the shared
+ * cache ([GIST 2.1, 2.3 item 1]: both views use one cache; [ABS]: O(1)
+ * overhead).  The pages leave the projections' epilogue open; this applies the
+ * Qwen3 family's: for token i of sequence b at position p = L_b + i and every
+ * head's d values x,
+ *   q and k heads: x_c <- x_c / sqrt(mean_c x_c^2 + rms_eps) * w_c  (skipped
+ *                  when both weights are NULL), then the rotary embedding
+ *                  y_j = x_j cos a_j - x_{j+d/2} sin a_j,
+ *                  y_{j+d/2} = x_{j+d/2} cos a_j + x_j sin a_j,
+ *                  a_j = p * rope_theta^(-2j/d) (angles in double precision);
+ *   v heads:       copied.
+ *   qkv         bf16 [B*K, (Hq + 2 Hkv) d] device, row = token b*K + i, heads
+ *               packed q (Hq) | k (Hkv) | v (Hkv)
+ *   q_norm_w, k_norm_w  bf16 [d] device, both or neither
+ *   rope_theta  > 0; rms_eps >= 0
+ *   Hq, K       query heads (multiple of cache->Hkv), block tokens (>= 1)
+ *   cache       KV cache view: k/v[b, g, L_b + i, :] receive the rotated k
+ *               and the v of KV head g; other slots are untouched
+ *   q_out       bf16 [B, K, Hq, d] device: the rotated queries, the layout
+ *               orthrus_block_attn reads
+ *   dev_status  int32 device or NULL: ORTHRUS_ECAPACITY when L_b + K > cap (L_b
+ *               is then clamped to cap - K, exactly as orthrus_block_attn does)
+ * Supported: d in {64, 128}.  Pointers 16-byte aligned.  No workspace.
+ */
+int orthrus_block_qkv_append(const void *qkv, const void *q_norm_w, const void *k_norm_w,
+                             float rope_theta, float rms_eps, int Hq, int K,
+                             const orthrus_kv_cache *cache, void *q_out, int32_t *dev_status,
+                             void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,8 @@ def load(path: str | None = None):
             "orthrus_verify": ([V, V, I, I, V, V, V], I),
             "orthrus_kv_commit": ([PC, V, I, V, V], I),
             "orthrus_verify_commit": ([V, V, I, I, V, V, PC, V, V], I),
+            "orthrus_block_qkv_append": ([V, V, V, ctypes.c_float, ctypes.c_float, I, I, PC,
+                                          V, V, V], I),
         }
         for name, (args, res) in sig.items():
             f = getattr(lib, name)
@@ -275,3 +277,31 @@ def verify_commit(argmax, draft, ctx_lens, cap: int, accept_len=None, next_tok=N
                                         _ptr(next_tok), ctypes.byref(view), _ptr(dev_status),
                                         _stream(stream)), "orthrus_verify_commit")
     return accept_len, next_tok
+
+
+def block_qkv_append(qkv, k_cache, v_cache, ctx_lens, Hq: int, K: int, q_norm_w=None,
+                     k_norm_w=None, rope_theta: float = 1e6, rms_eps: float = 1e-6,
+                     q_out=None, dev_status=None, stream=None,
+                     cache_view: KVCacheView | None = None):
+    """Per-head RMS norm of q/k, rotary embedding at L_b + i, block K/V into cache
+    slots [L_b, L_b + K): qkv bf16 [B*K, (Hq + 2 Hkv) d] -> q_out bf16 [B, K, Hq, d]."""
+    _need(qkv, torch.bfloat16, "qkv", 2)
+    view = cache_view if cache_view is not None else kv_cache_view(k_cache, v_cache, ctx_lens)
+    B, d = view.B, view.d
+    if qkv.shape != (B * K, (Hq + 2 * view.Hkv) * d):
+        raise ValueError("qkv must be [B*K, (Hq + 2 Hkv) d]")
+    for w, name in ((q_norm_w, "q_norm_w"), (k_norm_w, "k_norm_w")):
+        if w is not None:
+            _need(w, torch.bfloat16, name, 1)
+    if q_out is None:
+        q_out = torch.empty(B, K, Hq, d, dtype=torch.bfloat16, device=qkv.device)
+    else:
+        _need(q_out, torch.bfloat16, "q_out", 4)
+    if dev_status is not None:
+        _need(dev_status, torch.int32, "dev_status")
+    rc = load().orthrus_block_qkv_append(_ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w),
+                                         float(rope_theta), float(rms_eps), int(Hq), int(K),
+                                         ctypes.byref(view), _ptr(q_out), _ptr(dev_status),
+                                         _stream(stream))
+    _check(rc, "orthrus_block_qkv_append")
+    return q_out

@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
     for want in ("orthrus_block_attn", "orthrus_lmhead_argmax", "orthrus_verify",
                  "orthrus_kv_commit", "orthrus_verify_commit", "orthrus_row_argmax_f32",
                  "orthrus_block_attn_workspace_size", "orthrus_lmhead_workspace_size",
-                 "orthrus_status_str", "orthrus_abi_version"):
+                 "orthrus_status_str", "orthrus_abi_version", "orthrus_block_qkv_append"):
         assert want in names
 
 
@@ -116,3 +116,22 @@ def test_binding_refuses_cpu_tensors(lib):
     q = torch.zeros(1, 8, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ob.block_attn(q, q, q, torch.zeros(1, dtype=torch.int32), ob.MASK_AR)
+
+
+def test_qkv_append_host_validation(lib):
+    f = lib.orthrus_block_qkv_append
+    view = _view(B=2, Hkv=2, cap=64, d=128)
+    args = lambda **kw: (kw.get("qkv", A), kw.get("qw", None), kw.get("kw", None),
+                         kw.get("theta", 1e6), kw.get("eps", 1e-6), kw.get("Hq", 4),
+                         kw.get("K", 8), ctypes.byref(kw.get("view", view)), kw.get("out", A),
+                         None, None)
+    assert f(*args(qkv=None)) == ob.EINVAL
+    assert f(*args(K=0)) == ob.EINVAL
+    assert f(*args(theta=0.0)) == ob.EINVAL
+    assert f(*args(eps=-1.0)) == ob.EINVAL
+    assert f(*args(qw=A)) == ob.EINVAL                     # one weight without the other
+    assert f(*args(Hq=3)) == ob.ESHAPE
+    assert f(*args(view=_view(B=2, Hkv=2, cap=64, d=96))) == ob.EUNSUPPORTED
+    assert f(*args(K=65)) == ob.ESHAPE                     # cap < K
+    assert f(*args(out=A + 2)) == ob.EALIGN
+    assert f(*args(view=_view(B=0, Hkv=2, cap=64, d=128))) == ob.OK
