@@ -102,6 +102,18 @@ const char *orthrus_status_str(int status);
 int orthrus_abi_version(void);
 
 /*
+ * Process-wide limit, in nanoseconds, after which a bounded wait inside any
+ * kernel of this library gives up: the kernel then stores ORTHRUS_ETIMEOUT in
+ * dev_status, lets its in-flight copies and MMAs finish, frees its tensor
+ * memory and returns (its outputs are then undefined, and an attention
+ * workspace must be zeroed again).  Read at every launch; 0 restores the
+ * default of 2 s.  The kernels' real waits take microseconds, so only a
+ * watchdog or a test of the timeout path needs another value.  Always
+ * returns ORTHRUS_OK.  (No counterpart in the method: failure handling.)
+ */
+int orthrus_set_wait_limit_ns(uint64_t ns);
+
+/*
  * Workspace bytes orthrus_block_attn needs on the CURRENT device for these
  * shapes (split-KV partial results; independent of the context lengths).
  * Returns ORTHRUS_OK and writes *bytes, or a validation error.
@@ -125,14 +137,17 @@ int orthrus_block_attn_workspace_size(int B, int Hq, int Hkv, int d, int K, size
  *   mask_mode  orthrus_mask_mode, optionally | ORTHRUS_ATTN_DETERMINISTIC
  *   out        bf16 [B, K, Hq, d] device
  *   workspace  device, >= orthrus_block_attn_workspace_size(...) bytes, zero
- *              filled before the first call.  Its head holds a grid-barrier
- *              counter and, per (sequence, KV head, head chunk) segment, a
- *              completion counter and a work-claim counter; each call advances
- *              them in a way the next call can rebase on (the completion
- *              counters by exactly 2^20, the grid counter by the grid size), so
- *              a workspace is zeroed once, not per call (zero it again after an
- *              ORTHRUS_ETIMEOUT, and before using it on a device with a
- *              different SM count).  The rest holds per-call partial results.
+ *              filled before the first call.  Its head (at a fixed place for
+ *              every shape) holds a grid-barrier counter and, per (sequence,
+ *              KV head, head chunk) segment, a completion counter and a
+ *              work-claim counter.  Every completed call leaves them in the
+ *              state the next call starts from (grid counter a multiple of the
+ *              grid size, completion counters multiples of 2^20, claim
+ *              counters 0; the comparisons survive 64-bit wrap-around), so a
+ *              workspace is zeroed once, not per call, and serves any sequence
+ *              of shapes whose size query it satisfies.  Zero it again after an
+ *              ORTHRUS_ETIMEOUT and before using it on a device with a
+ *              different SM count.  The rest holds per-call partial results.
  *              Calls that share a workspace must be stream-ordered.
  *   dev_status int32 device or NULL (see conventions; ORTHRUS_ECAPACITY when
  *              L_b + K > cap, in which case L_b is clamped to cap - K)
@@ -189,8 +204,8 @@ int orthrus_lmhead_argmax(const void *h, const void *W, int R, int H, int V, int
  *   - All calls share the array (it keeps the last call's contents; nothing
  *     in it has to start zeroed).  Calls that overlap on the GPU race: order
  *     them on one stream.
- *   - Returns ORTHRUS_EWORKSPACE, launching nothing, on a device with more
- *     than 256 SMs (the array's capacity).
+ *   - Works on devices with up to 256 SMs (the array's capacity); returns
+ *     ORTHRUS_EWORKSPACE, launching nothing, on a device with more.
  * Arguments as for orthrus_lmhead_argmax, without the workspace.
  */
 int orthrus_lmhead_argmax_noalloc(const void *h, const void *W, int R, int H, int V,

@@ -8,33 +8,49 @@
 // diffusion mode and [0, L_b + i + 1) in AR mode.
 //
 // Design (B200, sm_100a).  One KV head serves G = Hq/Hkv query heads, so the
-// G*K queries of a (sequence, KV head) pair are packed into one 128-row tile
-// (row r = i*Gc + hh) and every K/V byte is read from HBM once.  The work of
-// all (sequence, KV head) segments is cut into 64-key tiles and spread evenly
-// over a persistent grid of one CTA per SM (split-KV / flash-decoding); a
-// CTA's contiguous tile range may cross segment boundaries and then emits one
-// partial result per segment piece.  Per CTA (12 warps), each single-thread
-// role on its own ring so no wait of one stream stalls another:
-//   warp 0      TMA: Q tile per piece, K tile groups into a ring.
-//   warp 2      TMA: V tile groups into a ring;
-//               the whole warp also allocates and frees TMEM.
-//   warp 1      tcgen05 issuer for S = Q K^T into TMEM buffer j % 4.
-//   warp 3      tcgen05 issuer for O_w += P V (P from the same TMEM buffer,
-//               V read MN-major from shared memory).
-//   warps 4-11  two softmax warpgroups taking alternate tiles, one thread per
-//               row: S from TMEM, mask, online softmax in the exp2 domain
-//               against a running reference max (O in TMEM is rescaled only
-//               when the max grows by more than 2^8, exact because the final
-//               normaliser uses the same reference), P as bf16 back into the
-//               tile's TMEM buffer.  At the end
-//               of a piece group 0 merges both groups' (m, l, O) and writes the
-//               piece's partial result.
-// The kernel is launched cooperatively: after writing its partials every CTA
-// meets the others at a bounded grid barrier and then merges an equal share of
-// the output rows (log-sum-exp over each segment's pieces, bf16 output), so the
-// whole operation is one launch.
+// G*K queries of a (sequence b, KV head g, head chunk hc) segment are packed
+// into one 128-row tcgen05 M tile (row r = i*Gc + hh) and every K/V byte is
+// read from HBM once.  One cooperative, persistent launch of one CTA per SM;
+// the keys of each segment are cut into 64-key tiles, loaded in groups of two
+// (one 128-row TMA box per 128-byte column chunk).
+//
+// Partition.  When the segments fit the grid (S <= SMs) every CTA works
+// inside one segment: segment s gets CTAs in proportion to its tiles.  By
+// default a CTA streams a static run of about 3/4 of its fair share of the
+// segment's groups and then claims the rest one group at a time from the
+// segment's claim counter (dynamic balance: siblings finish within about one
+// group of each other); ORTHRUS_ATTN_DETERMINISTIC gives every CTA a fixed
+// range instead.  With more segments than CTAs the flat tile range is split
+// evenly (stream-K) and a CTA may cross segments, emitting one partial result
+// per segment piece.
+//
+// Roles (12 warps), each single-thread role on its own mbarrier ring:
+//   warp 0      computes the CTA's schedule from ctx_lens (lane-parallel
+//               scans), publishes the CTA's load groups as items of a ring
+//               in shared memory (every other role replays the same list),
+//               TMA-loads the Q tile of each piece and K into 3 stages.
+//   warp 2      TMA-loads V into 3 stages; the whole warp allocates and frees
+//               TMEM (all 512 columns).
+//   warp 1      tcgen05 issuer of S = Q K^T, one N = 128 sequence per group
+//               into one of two 128-column TMEM S buffers.
+//   warp 3      tcgen05 issuer of O_w += P V, P read from TMEM (the bf16 P of
+//               a tile overwrites its S columns), V an MN-major smem operand.
+//   warps 4-11  two softmax warpgroups on alternate tiles, one thread per
+//               row: S from TMEM, tail masking only on tail tiles, exp2
+//               against a running reference max (O is rescaled only when the
+//               max grows by more than 2^8, exact because the final
+//               normaliser uses the same reference), P back into TMEM.  At a
+//               piece end the two groups merge their (m, l, O) and write the
+//               piece's fp32 partial result.
+// Merge.  Per-segment partition: each CTA adds to its segment's completion
+// counter once its partial is written; the segment's own CTAs then fold an
+// equal share of its rows by log-sum-exp (bulk copies of the pieces' rows
+// into the idle K/V ring) and write bf16.  Stream-K: a bounded grid barrier,
+// then every CTA merges an equal share of all output rows.  The whole
+// operation is one launch.
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <cmath>
 
 #include "common.cuh"
@@ -89,7 +105,7 @@ struct Layout {
   static constexpr int OFF_SCHED = OFF_ML + ROWS * 8;  // 9 x int64 CTA schedule
   static constexpr int OFF_ITEMS = OFF_SCHED + 128;  // RING x int4 work items
   static constexpr int OFF_BAR = OFF_ITEMS + RING * 16;
-  static constexpr int NBAR = 2 * NK + 2 * NV + 13 + RING;
+  static constexpr int NBAR = 2 * NK + 2 * NV + 15 + RING;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
@@ -103,10 +119,11 @@ struct Params {
   float* part_o;      // [slots][ROWS][D] unnormalised O of each piece
   float2* part_ml;    // [slots][ROWS] (m in log2 units, l)
   unsigned long long* gbar;  // grid-barrier arrival ticket counter (starts at 0)
-  unsigned long long* seg_cnt;  // [S] per-segment completion counters (start at 0)
-  unsigned long long* seg_next; // [S] per-segment group claim counters (start at 0)
+  unsigned long long* seg_cnt;  // [SMs] per-segment completion counters (start at 0)
+  unsigned long long* seg_next; // [SMs] per-segment group claim counters (0 between calls)
   __nv_bfloat16* out; // [B, K, Hq, D]
   int32_t* dev_status;
+  unsigned long long wait_ns;  // bounded-wait limit
   int B, K, Hq, Hkv, G, Gc, nhc, cap, mask_mode;
   int balance;        // per-segment partition: claim the tail groups dynamically
   float sl2;          // softmax scale * log2(e)
@@ -230,12 +247,12 @@ __device__ __forceinline__ void write_sched(long long* sched, int x0, int x1, in
   sched[8] = (static_cast<long long>(L) << 32) | static_cast<unsigned int>(nb);
 }
 
+// `raw` is lane b's ctx_lens[b] (0 for lanes >= B).
 __device__ void warp_schedule_small(const Params& p, int P, int c, int lane, bool report_errors,
-                                    long long* sched) {
+                                    long long* sched, int raw) {
   const int nseg = p.Hkv * p.nhc;
   const int S = p.B * nseg;
   const bool in = lane < p.B;
-  const int raw = in ? __ldg(p.ctx_lens + lane) : 0;
   if (report_errors && in && (raw < 0 || raw > p.cap - p.K)) report(p.dev_status, ORTHRUS_ECAPACITY);
   const int L = in ? clamp_len(raw, p) : 0;
   const int nb = in ? n_tiles(L, p) : 0;
@@ -299,7 +316,8 @@ __device__ void warp_schedule_small(const Params& p, int P, int c, int lane, boo
 __device__ void warp_schedule(const Params& p, int P, int c, int lane, bool report_errors,
                               long long* sched) {
   if (p.B <= 32) {
-    warp_schedule_small(p, P, c, lane, report_errors, sched);
+    warp_schedule_small(p, P, c, lane, report_errors, sched,
+                        lane < p.B ? __ldcg(p.ctx_lens + lane) : 0);
     return;
   }
   const int nseg = p.Hkv * p.nhc;
@@ -402,6 +420,8 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
 // nctas per launch (so it stays a multiple of nctas between launches and
 // never needs resetting); the generation is complete once the counter reaches
 // the next multiple.  Bounded: a wait that gives up reports ETIMEOUT.
+// grid_wait compares by signed difference, so a counter that wraps past 2^64
+// still reaches its target.
 __device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* gbar,
                                                           unsigned int nctas) {
   __threadfence();
@@ -409,17 +429,20 @@ __device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* gb
   return (ticket / nctas + 1) * nctas;
 }
 
-__device__ void grid_wait(unsigned long long* gbar, unsigned long long target,
-                          int32_t* status) {
+__device__ bool grid_wait(unsigned long long* gbar, unsigned long long target,
+                          int32_t* status, uint64_t limit_ns) {
   volatile unsigned long long* v = gbar;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t polls = 0; *v < target; ++polls) {
-    if ((polls & 255u) == 255u && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+  bool ok = true;
+  for (uint32_t polls = 0; static_cast<long long>(*v - target) < 0; ++polls) {
+    if ((polls & 255u) == 255u && globaltimer_ns() - t0 > limit_ns) {
       report(status, ORTHRUS_ETIMEOUT);
+      ok = false;
       break;
     }
   }
   __threadfence();
+  return ok;
 }
 
 // CTAs [*c0, *c1] may hold pieces of segment s = (b, seg); *tall is the flat
@@ -567,7 +590,7 @@ __device__ void merge_rows(const Params& p, int P, long long r0, long long r1, i
 // batch into its running (M, L, acc) -- every thread of a row derives the
 // same weights from the shared (m, l) table -- and finally writes acc / L as
 // bf16.  `buf` is the idle K/V ring (1024-aligned).
-template <int D>
+template <int D, bool kShortWait>
 __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int row1, int warp,
                               int lane, uint8_t* buf, volatile int* abort_flag) {
   constexpr int RC = 8;                                  // rows per round
@@ -587,6 +610,12 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
     fence_mbar_init();
   }
   __syncthreads();
+  // A wait of this CTA gave up: the status is set and nothing is merged.  The
+  // second barrier keeps a later wait from raising the flag before every
+  // thread has read it.
+  const bool skip = *abort_flag != 0;
+  __syncthreads();
+  if (skip) return;
   const bool dense = p.balance || own.cn <= own.ns;  // every CTA wrote a (maybe empty) piece
   auto live = [&](int j) {
     return dense || mul_div(j, own.ns, own.cn) != mul_div(j + 1, own.ns, own.cn);
@@ -627,9 +656,13 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
         ml_s[t] = (r < nr && live(j0 + jj)) ? __ldcg(p.part_ml + slot * ROWS + rb + r)
                                             : make_float2(-INFINITY, 0.f);
       }
-      mbar_wait_bounded(bar, phase, abort_flag, p.dev_status);  // gives up: status set
+      // A wait that gives up still lets this round's copies land before the
+      // CTA leaves (they target its shared memory); then every thread returns.
+      if (!mbar_wait_bounded<kShortWait>(bar, phase, abort_flag, p.dev_status, p.wait_ns))
+        mbar_wait_drain(bar, phase, p.dev_status);
       phase ^= 1u;
       __syncthreads();
+      if (*abort_flag) return;  // read by all threads between the same two barriers
       if (tr < nr) {
         float mb = M;
         for (int jj = 0; jj < nb; ++jj) mb = fmaxf(mb, ml_s[jj * RC + tr].x);
@@ -673,7 +706,7 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
   }
 }
 
-template <int D>
+template <int D, bool kShortWait>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_splitkv_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK2,
@@ -706,17 +739,33 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t o_full = bar2 + 8u * 10;
   const uint32_t o_free = bar2 + 8u * 11;
   const uint32_t mma_done = bar2 + 8u * 12;  // both MMA issuers commit once at exit
-  auto item_full = [&](int i) { return bar2 + 8u * (13 + i); };  // work item i published
+  // piece epilogue hand-offs between the softmax groups (bounded waits, so a
+  // group that gave up never leaves the other one stuck at a barrier)
+  const uint32_t xchg_ml = bar2 + 8u * 13;      // WG1's (m, l) are in ml_xchg
+  const uint32_t xchg_scale = bar2 + 8u * 14;   // WG0's two scales are in ml_xchg
+  auto item_full = [&](int i) { return bar2 + 8u * (15 + i); };  // work item i published
   int4* items = reinterpret_cast<int4*>(smem + Ly::OFF_ITEMS);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly::OFF_MISC + 4);
   float2* ml_xchg = reinterpret_cast<float2*>(smem + Ly::OFF_ML);
 
-  // The CTA's tile range and its starting cursor are computed once, by
-  // thread 0, and shared.
+  // Programmatic dependent launch: the next kernel in the stream may be
+  // scheduled now (its CTAs land on SMs as this grid's CTAs exit).  Until
+  // grid_dep_wait below this kernel touches only its own shared and tensor
+  // memory, L2 prefetches and ctx_lens, which it reads speculatively (through
+  // L2, never L1) and reads again after the wait.
+  grid_dep_launch();
+
+  // The CTA's tile range and its starting cursor are computed by warp 0 and
+  // shared.  With up to 32 sequences a speculative schedule from the lengths
+  // as they stand is computed before the dependency wait and kept if the
+  // lengths read after the wait are the same.
   long long* sched = reinterpret_cast<long long*>(smem + Ly::OFF_SCHED);
-  if (warp == 0) {
-    warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
+  const bool spec = p.B <= 32;
+  int spec_raw = 0;
+  if (warp == 0 && spec) {
+    spec_raw = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
+    warp_schedule_small(p, gridDim.x, blockIdx.x, lane, false, sched, spec_raw);
     __syncwarp();
   }
 
@@ -753,7 +802,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   int pr_n = 0, pr_j = 0, pr_cur = -2;
   int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0;
   bool pr_grabbing = false, pr_dry = true;
-  unsigned long long pr_base = 0, pr_pend = 0;
+  unsigned long long pr_pend = 0;
   const uint64_t pr_policy = policy_evict_first();
   int pr_s = -1, pr_kvbase = 0, pr_qh = 0, pr_qb = 0;  // cached for the current segment
   auto emit = [&](int t, int L, int s, int flags) -> bool {
@@ -774,7 +823,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_arrive(item_full(slot));
     if (flags & kItemNone) return true;
     if (flags & kItemPieceFirst) {
-      if (!mbar_wait_bounded(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status)) return false;
+      if (!mbar_wait_bounded<kShortWait>(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status, p.wait_ns))
+        return false;
       mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.Gc * p.K * D * 2));
       for (int c = 0; c < Ly::CHUNKS; ++c)
         tma_load_3d(sb0 + Ly::OFF_Q + c * Ly::Q_CHUNK, &tmQ, q_full, c * 64, pr_qh, pr_qb);
@@ -782,7 +832,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const bool pair = flags & kItemPair;
     const int stage = pr_gi % NK;
-    if (!mbar_wait_bounded(empty_k(stage), ((pr_gi / NK) & 1) ^ 1, abort_flag, p.dev_status))
+    if (!mbar_wait_bounded<kShortWait>(empty_k(stage), ((pr_gi / NK) & 1) ^ 1, abort_flag, p.dev_status,
+                           p.wait_ns))
       return false;
     mbar_arrive_expect_tx(full_k(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
     for (int c = 0; c < Ly::CHUNKS; ++c)
@@ -795,15 +846,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   // about 3/4 of its fair share of the segment's 128-key groups, then claims
   // groups of the remaining pool one at a time from the segment's claim
   // counter (the next claim is always in flight, so its latency is hidden,
-  // and siblings finish within about one group of each other).  The
-  // counter is rebased per call to epoch E << 32, E being the number of
-  // completed calls read from the segment's completion counter (which cannot
-  // reach the next multiple of 2^20 before this CTA's own add).
+  // and siblings finish within about one group of each other).  The counter
+  // is 0 when a call starts: the segment's last CTA puts it back to 0 once
+  // every sibling has finished claiming (see the merge below).
   auto start_claims = [&]() {
-    const unsigned long long done =
-        *reinterpret_cast<volatile unsigned long long*>(p.seg_cnt + pr_own.s);
-    pr_base = (done >> 20) << 32;
-    atomicMax(p.seg_next + pr_own.s, pr_base);
     pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);
     pr_grabbing = true;
   };
@@ -815,7 +861,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (pr_dry) return -1;
     if (!pr_grabbing) start_claims();
-    const long long g = pr_pool0 + static_cast<long long>(pr_pend - pr_base);
+    const long long g = pr_pool0 + static_cast<long long>(pr_pend);
     if (g >= pr_ngr) {
       pr_dry = true;
       return -1;
@@ -887,23 +933,35 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(o_full, 1);
     mbar_init(o_free, 8);
     mbar_init(mma_done, 2);
+    mbar_init(xchg_ml, 4);
+    mbar_init(xchg_scale, 4);
     for (int i = 0; i < RING; ++i) mbar_init(item_full(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // warp 0 wrote the schedule (the warp converged after warp_schedule)
-    pr_own = read_own();
-    pr_c = read_start();
-    pr_n = static_cast<int>(sched[1] - sched[0]);
-    if (pr_own.s >= 0 && p.balance) {
-      const int k = static_cast<int>(blockIdx.x) - pr_own.c0;
-      pr_ngr = (pr_own.ns + 1) / 2;
-      const int fs = static_cast<int>(mul_div(3 * pr_ngr, 1, 4 * pr_own.cn));
-      pr_pool0 = pr_own.cn * fs;
-      pr_sg = k * fs;
-      pr_sg_end = pr_sg + fs;
-      pr_dry = pr_pool0 >= pr_ngr;
+    if (spec) {
+      // Warm L2 with the first groups of the speculative schedule while the
+      // previous kernel finishes (a stale schedule only wastes the prefetch).
+      prefetch_tmap(&tmK2);
+      prefetch_tmap(&tmV2);
+      const OwnSeg o = read_own();
+      if (o.s >= 0) {
+        const int b = static_cast<int>(o.s / nseg), seg = static_cast<int>(o.s % nseg);
+        const int kvbase = (b * p.Hkv + seg / p.nhc) * p.cap;
+        int t0 = static_cast<int>(sched[4] >> 32), t1 = t0 + static_cast<int>(sched[1] - sched[0]);
+        if (p.balance) {
+          const int ngr = (o.ns + 1) / 2;
+          const int fs = static_cast<int>(mul_div(3 * ngr, 1, 4 * o.cn));
+          t0 = 2 * (static_cast<int>(blockIdx.x) - o.c0) * fs;
+          t1 = t0 + 2 * fs;
+        }
+        if (t1 > t0 + 2 * NK) t1 = t0 + 2 * NK;
+        for (int t = t0; t < t1; t += 2)
+          for (int c = 0; c < Ly::CHUNKS; ++c) {
+            tma_prefetch_2d(&tmK2, c * 64, kvbase + t * TN);
+            tma_prefetch_2d(&tmV2, c * 64, kvbase + t * TN);
+          }
+      }
     }
-    produce(NK, true);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -922,15 +980,47 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     fence_proxy_async_smem();
   }
+
+  // Everything a preceding kernel may write (ctx_lens, q, the cache, the
+  // workspace, dev_status) is read or written only after this point.
+  grid_dep_wait();
+  if (warp == 0) {
+    if (spec) {
+      const int raw = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
+      if (!__all_sync(0xFFFFFFFFu, raw == spec_raw))
+        warp_schedule_small(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched, raw);
+      else if (blockIdx.x == 0 && lane < p.B && (raw < 0 || raw > p.cap - p.K))
+        report(p.dev_status, ORTHRUS_ECAPACITY);
+    } else {
+      warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
+    }
+    __syncwarp();
+  }
+  if (threadIdx.x == 0) {
+    // warp 0 wrote the schedule (the warp converged after it)
+    pr_own = read_own();
+    pr_c = read_start();
+    pr_n = static_cast<int>(sched[1] - sched[0]);
+    if (pr_own.s >= 0 && p.balance) {
+      const int k = static_cast<int>(blockIdx.x) - pr_own.c0;
+      pr_ngr = (pr_own.ns + 1) / 2;
+      const int fs = static_cast<int>(mul_div(3 * pr_ngr, 1, 4 * pr_own.cn));
+      pr_pool0 = pr_own.cn * fs;
+      pr_sg = k * fs;
+      pr_sg_end = pr_sg + fs;
+      pr_dry = pr_pool0 >= pr_ngr;
+    }
+    produce(NK, true);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
 #define WAIT_OR(barrier, parity, on_fail) \
-  if (!mbar_wait_bounded((barrier), (parity), abort_flag, p.dev_status)) on_fail
+  if (!mbar_wait_bounded<kShortWait>((barrier), (parity), abort_flag, p.dev_status, p.wait_ns)) on_fail
 #define WARP_WAIT_OR(barrier, parity, on_fail) \
-  if (!mbar_wait_warp((barrier), (parity), abort_flag, p.dev_status)) on_fail
+  if (!mbar_wait_warp<kShortWait>((barrier), (parity), abort_flag, p.dev_status, p.wait_ns)) on_fail
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------ work list, Q and K producer
@@ -1090,7 +1180,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     // O through 0 * NaN.  Returns false if the V stage never arrived.
     auto zero_v_tail = [&](int tile0, int kv_end, bool first_half) -> bool {
       const int stage = gi % NV;
-      if (!mbar_wait_warp(full_v(stage), (gi / NV) & 1, abort_flag, p.dev_status)) return false;
+      if (!mbar_wait_warp<kShortWait>(full_v(stage), (gi / NV) & 1, abort_flag, p.dev_status, p.wait_ns))
+        return false;
       const int nv = kv_end - tile0 > 0 ? kv_end - tile0 : 0;
       const int per_chunk = (TN - nv) * 8;
       uint8_t* vt = smem + Ly::OFF_V + stage * Ly::KV_BYTES + (first_half ? 0 : Ly::HALF);
@@ -1249,28 +1340,33 @@ __global__ void __launch_bounds__(THREADS, 1)
 
       if (flags & kItemPieceLast) {
         // Piece epilogue: merge the two groups' (m, l, O) and publish it.  WG1
-        // hands its (m, l) to WG0, which writes the row's (M, l) and hands
-        // back the two scales; then each group writes half of the columns.
+        // hands its (m, l) to WG0 (xchg_ml), which writes the row's (M, l) and
+        // hands back the two scales in the same slot (xchg_scale); then each
+        // group writes half of the columns.  Thread r of each group is the
+        // only reader and writer of ml_xchg[r] on its side, and each side
+        // writes only after the other side's hand-off, so one slot suffices.
         WARP_WAIT_OR(o_full, pieces & 1, break);
         tc_fence_after();
         const long long pslot = static_cast<long long>(items[slot].z) + blockIdx.x;
-        if (w == 1) ml_xchg[r] = make_float2(m_used, l_sum);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
         float a0, a1;
-        if (w == 0) {
+        if (w == 1) {
+          ml_xchg[r] = make_float2(m_used, l_sum);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xchg_ml);
+          WARP_WAIT_OR(xchg_scale, pieces & 1, break);
+          const float2 sc = ml_xchg[r];
+          a0 = sc.x;
+          a1 = sc.y;
+        } else {
+          WARP_WAIT_OR(xchg_ml, pieces & 1, break);
           const float2 o1 = ml_xchg[r];
           const float M = fmaxf(m_used, o1.x);
           a0 = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - M);
           a1 = (o1.x == -INFINITY) ? 0.f : fast_exp2(o1.x - M);
           if (!idle_warp) p.part_ml[pslot * ROWS + r] = make_float2(M, a0 * l_sum + a1 * o1.y);
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (w == 0) ml_xchg[r] = make_float2(a0, a1);
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (w == 1) {
-          const float2 sc = ml_xchg[r];
-          a0 = sc.x;
-          a1 = sc.y;
+          ml_xchg[r] = make_float2(a0, a1);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xchg_scale);
         }
         if (!idle_warp) {  // rows of all-padding warps are never merged
           float* dst = p.part_o + (pslot * ROWS + r) * D;
@@ -1322,7 +1418,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // segment's counter once their piece is written (the first adds 2^20 -
     // (cn - 1), the rest 1, so every call adds exactly 2^20 and the counter
     // never needs a reset); a CTA's own add pins the call's target.  Then the
-    // segment's rows are merged by its own CTAs, an equal share each.
+    // segment's rows are merged by its own CTAs, an equal share each.  All
+    // siblings have added only after their last claim, so once the target is
+    // reached the last CTA of the segment (which always has rows to merge)
+    // puts the claim counter back to 0 for the next call.
     const int k = static_cast<int>(blockIdx.x) - own.c0;
     const int row0 = static_cast<int>(mul_div(k, RV, own.cn));
     const int row1 = static_cast<int>(mul_div(k + 1, RV, own.cn));
@@ -1330,10 +1429,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       __threadfence();
       const unsigned long long add = k == 0 ? (1ull << 20) - (own.cn - 1) : 1ull;
       const unsigned long long old = atomicAdd(p.seg_cnt + own.s, add);
-      if (row1 > row0) grid_wait(p.seg_cnt + own.s, ((old >> 20) + 1) << 20, p.dev_status);
+      if (row1 > row0 &&
+          grid_wait(p.seg_cnt + own.s, ((old >> 20) + 1) << 20, p.dev_status, p.wait_ns) &&
+          k == own.cn - 1 && p.balance)
+        *reinterpret_cast<volatile unsigned long long*>(p.seg_next + own.s) = 0ull;
     }
     __syncthreads();
-    merge_segment<D>(p, own, row0, row1, warp, lane, smem + Ly::OFF_K, abort_flag);
+    merge_segment<D, kShortWait>(p, own, row0, row1, warp, lane, smem + Ly::OFF_K, abort_flag);
     return;
   }
 
@@ -1351,7 +1453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     const unsigned long long target = grid_arrive(p.gbar, gridDim.x);
     for (int k = 0; k < n_segs; ++k) segs[k] = segment_pieces(p, gridDim.x, s_first + k);
-    grid_wait(p.gbar, target, p.dev_status);
+    grid_wait(p.gbar, target, p.dev_status, p.wait_ns);
   }
   __syncthreads();
   merge_rows<D>(p, gridDim.x, r0, r1, warp, THREADS / 32, lane, segs, s_first, n_segs);
@@ -1379,21 +1481,26 @@ int check_shape(int B, int Hq, int Hkv, int d, int K, Shape* sh) {
   return ORTHRUS_OK;
 }
 
-// Workspace: [0, 256) the grid-barrier ticket, then one 64-bit completion
-// counter per segment (padded to 256 bytes), then the partial O and (m, l) of
-// every piece.  The counters must be zero before the first use; every call
-// advances them by fixed amounts, so they never need resetting.
+// Workspace: [0, 256) the grid-barrier ticket, then `sms` 64-bit completion
+// counters and `sms` 64-bit claim counters (per-segment counters exist only
+// when the segments fit the grid, S <= sms, so this region has the same size
+// and place for every shape), padded to 256 bytes, then the partial O and
+// (m, l) of every piece.  The counters must be zero before the first use;
+// after every completed call the ticket is a multiple of the grid size, each
+// completion counter a multiple of 2^20 and each claim counter 0, whatever
+// the shape, so one zeroed workspace serves any sequence of shapes it is large
+// enough for.
 constexpr size_t WS_TICKET = 256;
 
-size_t counter_bytes(const Shape& sh) {  // completion + claim counters
-  return (2 * static_cast<size_t>(sh.S) * sizeof(unsigned long long) + 255) / 256 * 256;
+size_t counter_bytes(int sms) {  // completion + claim counters
+  return (2 * static_cast<size_t>(sms) * sizeof(unsigned long long) + 255) / 256 * 256;
 }
 
 size_t workspace_bytes(const Shape& sh, int sms) {
   const size_t slots = static_cast<size_t>(sh.S) + static_cast<size_t>(sms);
   const size_t o_bytes = slots * ROWS * sh.d * sizeof(float);
   const size_t ml_bytes = slots * ROWS * sizeof(float2);
-  return WS_TICKET + counter_bytes(sh) + o_bytes + ml_bytes;
+  return WS_TICKET + counter_bytes(sms) + o_bytes + ml_bytes;
 }
 
 template <int D>
@@ -1428,12 +1535,13 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.gbar = reinterpret_cast<unsigned long long*>(w);
   p.seg_cnt = reinterpret_cast<unsigned long long*>(w + WS_TICKET);
-  p.seg_next = p.seg_cnt + sh.S;
-  const size_t head = WS_TICKET + counter_bytes(sh);
+  p.seg_next = p.seg_cnt + sms;
+  const size_t head = WS_TICKET + counter_bytes(sms);
   p.part_o = reinterpret_cast<float*>(w + head);
   p.part_ml = reinterpret_cast<float2*>(w + head + slots * ROWS * D * sizeof(float));
   p.out = static_cast<__nv_bfloat16*>(out);
   p.dev_status = dev_status;
+  p.wait_ns = wait_limit_ns();
   p.B = sh.B;
   p.K = sh.K;
   p.Hq = sh.Hq;
@@ -1446,22 +1554,37 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   p.balance = (mask_mode & ORTHRUS_ATTN_DETERMINISTIC) ? 0 : 1;
   p.sl2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
 
-  auto* kfn = attn_splitkv_kernel<D>;
+  auto* kfn = p.wait_ns < kShortWaitNs ? attn_splitkv_kernel<D, true>
+                                       : attn_splitkv_kernel<D, false>;
   if (!opt_in_smem(reinterpret_cast<const void*>(kfn), Layout<D>::ALLOC)) return ORTHRUS_ECUDA;
   // Cooperative launch: the grid barrier before the merge needs every CTA
-  // resident at once (one CTA per SM).
+  // resident at once (one CTA per SM).  Programmatic stream serialisation lets
+  // the kernel's prologue overlap the tail of the previous kernel in the
+  // stream; the kernel waits (griddepcontrol.wait) before it reads anything
+  // that kernel may have written.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = Layout<D>::ALLOC;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p) != cudaSuccess)
-    return ORTHRUS_ECUDA;
+  // If the runtime refuses the pair of attributes, the first (eager) call
+  // finds out and every later call launches cooperatively only.
+  static std::atomic<bool> coop_pdl_ok{true};
+  cfg.numAttrs = (pdl_enabled() && coop_pdl_ok.load(std::memory_order_relaxed)) ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
+  if (e != cudaSuccess && cfg.numAttrs == 2) {
+    (void)cudaGetLastError();
+    coop_pdl_ok.store(false, std::memory_order_relaxed);
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
+  }
+  if (e != cudaSuccess) return ORTHRUS_ECUDA;
   return ORTHRUS_OK;
 }
 

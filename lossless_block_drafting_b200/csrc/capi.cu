@@ -2,6 +2,8 @@
 // queries shared by the kernels' host launchers.
 #include <cudaTypedefs.h>
 
+#include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 #include "host.h"
@@ -65,6 +67,18 @@ bool opt_in_smem(const void* kernel, int bytes) {
   return true;
 }
 
+namespace {
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s
+std::atomic<uint64_t> g_wait_ns{kDefaultWaitNs};
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
+
+bool pdl_enabled() {
+  static const bool on = std::getenv("ORTHRUS_NO_PDL") == nullptr;
+  return on;
+}
+
 int current_sm_count(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;
@@ -90,4 +104,9 @@ extern "C" const char* orthrus_status_str(int status) {
   }
 }
 
-extern "C" int orthrus_abi_version(void) { return 1; }
+extern "C" int orthrus_abi_version(void) { return 2; }
+
+extern "C" int orthrus_set_wait_limit_ns(uint64_t ns) {
+  orthrus::g_wait_ns.store(ns == 0 ? orthrus::kDefaultWaitNs : ns, std::memory_order_relaxed);
+  return ORTHRUS_OK;
+}

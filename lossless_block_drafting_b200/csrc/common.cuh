@@ -8,9 +8,9 @@
 
 namespace orthrus {
 
-// A bounded wait gives up after this long (the kernels' real waits take
+// A bounded wait gives up after `limit_ns` (the launch's wait limit: 2 s unless
+// orthrus_set_wait_limit_ns changed it; the kernels' real waits take
 // microseconds); the CTA then records ORTHRUS_ETIMEOUT and unwinds.
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitMaxPolls = 1u << 30;
 
 // Store `code` into *status if it is still 0 (first error wins).
@@ -18,20 +18,47 @@ __device__ __forceinline__ void report(int32_t* status, int code) {
   if (status != nullptr) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
+// Limits below this select the kernels' short-wait instantiation (a watchdog
+// or a test of the timeout path); the common path never pays for it.
+constexpr uint64_t kShortWaitNs = 1000000ull;  // 1 ms
+
 // Wait for the phase of `bar` with the given parity.  Returns false if the
-// CTA-wide abort flag is raised or the wait runs out of time (which raises it).
+// CTA-wide abort flag is raised or the wait runs out of time (which raises
+// it).
+//   kShort = false: one try_wait is the common path (it suspends the thread
+//     until the phase completes or a hardware window ends); the abort flag and
+//     the clock are looked at every 32 polls.
+//   kShort = true (limit_ns < kShortWaitNs): every try_wait suspends the
+//     thread for at most limit_ns, and flag and clock are looked at after
+//     each, so the limit is noticed even when no hardware window would
+//     outlast it.
+template <bool kShort>
 static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t polls = 1;; ++polls) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((polls & 31u) == 0) {
+                                                      volatile int* abort_flag, int32_t* status,
+                                                      uint64_t limit_ns) {
+  if constexpr (kShort) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t polls = 0;; ++polls) {
+      if (mbar_try_wait_for(bar, parity, static_cast<uint32_t>(limit_ns))) return true;
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs || polls > kWaitMaxPolls) {
+      if (globaltimer_ns() - t0 > limit_ns || polls > kWaitMaxPolls) {
         *abort_flag = 1;
         report(status, ORTHRUS_ETIMEOUT);
         return false;
+      }
+    }
+  } else {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t polls = 1;; ++polls) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((polls & 31u) == 0) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns || polls > kWaitMaxPolls) {
+          *abort_flag = 1;
+          report(status, ORTHRUS_ETIMEOUT);
+          return false;
+        }
       }
     }
   }
@@ -40,10 +67,12 @@ static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t par
 // Warp-collective variant: every lane waits, and the warp proceeds only if all
 // lanes succeeded, so warp-wide tcgen05 instructions after it are never
 // reached by part of a warp.
+template <bool kShort>
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
-                                               volatile int* abort_flag, int32_t* status) {
-  if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;  // common case
-  const bool ok = mbar_wait_bounded(bar, parity, abort_flag, status);
+                                               volatile int* abort_flag, int32_t* status,
+                                               uint64_t limit_ns) {
+  if (!kShort && __all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;  // common case
+  const bool ok = mbar_wait_bounded<kShort>(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xFFFFFFFFu, ok);
 }
 

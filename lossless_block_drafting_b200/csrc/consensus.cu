@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(WARPS * 32)
     verify_commit_kernel(const int32_t* __restrict__ argmax, const int32_t* __restrict__ draft,
                          int B, int K, int32_t* accept_len, int32_t* next_tok,
                          int32_t* ctx_lens, int cap, int32_t* dev_status, int mode) {
+  grid_dep_launch();
+  grid_dep_wait();  // argmax, draft, accept_len and ctx_lens may come from the previous kernel
   const int b = blockIdx.x * WARPS + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -66,6 +68,8 @@ __global__ void __launch_bounds__(WARPS * 32)
 // Greedy choice over fp32 logits: one block per row, smallest index on ties.
 __global__ void __launch_bounds__(256) row_argmax_kernel(const float* __restrict__ logits, int V,
                                                          int32_t* __restrict__ argmax) {
+  grid_dep_launch();
+  grid_dep_wait();
   const int r = blockIdx.x;
   const float* row = logits + static_cast<long long>(r) * V;
   uint64_t k = 0ull;
@@ -87,9 +91,9 @@ int launch_vc(const int32_t* argmax, const int32_t* draft, int B, int K, int32_t
               void* stream) {
   if (B == 0) return ORTHRUS_OK;
   const int blocks = (B + WARPS - 1) / WARPS;
-  verify_commit_kernel<<<blocks, WARPS * 32, 0, as_stream(stream)>>>(
-      argmax, draft, B, K, accept_len, next_tok, ctx_lens, cap, dev_status, mode);
-  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+  return launch_kernel(verify_commit_kernel, dim3(blocks), dim3(WARPS * 32), 0, as_stream(stream),
+                       argmax, draft, B, K, accept_len, next_tok, ctx_lens, cap, dev_status,
+                       mode);
 }
 
 }  // namespace cons
@@ -136,6 +140,6 @@ extern "C" int orthrus_row_argmax_f32(const float* logits, int R, int V, int32_t
   if (R < 0 || V < 1) return ORTHRUS_EINVAL;
   if (R > 0 && (logits == nullptr || argmax == nullptr)) return ORTHRUS_EINVAL;
   if (R == 0) return ORTHRUS_OK;
-  cons::row_argmax_kernel<<<R, 256, 0, as_stream(stream)>>>(logits, V, argmax);
-  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+  return launch_kernel(cons::row_argmax_kernel, dim3(R), dim3(256), 0, as_stream(stream), logits,
+                       V, argmax);
 }

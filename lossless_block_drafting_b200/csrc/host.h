@@ -26,6 +26,34 @@ int current_sm_count(int* sms);
 // being captured into a CUDA graph issue no attribute call.
 bool opt_in_smem(const void* kernel, int bytes);
 
+// Limit, in nanoseconds, after which a bounded wait inside a kernel gives up
+// (passed to every launch; 2 s unless orthrus_set_wait_limit_ns changed it).
+uint64_t wait_limit_ns();
+
+// Whether launches carry the programmatic-stream-serialisation attribute
+// (on unless the environment variable ORTHRUS_NO_PDL is set when the library
+// first launches a kernel).
+bool pdl_enabled();
+
+// Launch `kernel` on `s`, with the programmatic-stream-serialisation
+// attribute when pdl_enabled(); every kernel of this library calls
+// griddepcontrol.wait before it touches memory a preceding kernel may write.
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                  Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }

@@ -41,6 +41,7 @@ constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in maximum per block
 struct Params {
   uint64_t* part_keys;  // [gridDim.x][Npad]
   int32_t* dev_status;
+  unsigned long long wait_ns;  // bounded-wait limit
   int R, Npad, H, V, TPR, NS, stage_bytes;
 };
 
@@ -70,6 +71,13 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
   }
 }
 
+// Rows of tile t of a CTA's vocabulary slice [row0, row_end).
+__device__ __forceinline__ int tile_rows_of(int row0, int row_end, int t) {
+  const int a = row0 + t * BM;
+  const int e = a + BM < row_end ? a + BM : row_end;
+  return e - a;
+}
+
 // 32 keys per lane -> lane l holds the warp-wide max of column l.
 __device__ __forceinline__ uint64_t transpose_max(uint64_t (&v)[32], int lane) {
 #pragma unroll
@@ -85,6 +93,7 @@ __device__ __forceinline__ uint64_t transpose_max(uint64_t (&v)[32], int lane) {
   return v[0];
 }
 
+template <bool kShortWait>
 __global__ void __launch_bounds__(THREADS, 1)
     lmhead_argmax_kernel(const __grid_constant__ CUtensorMap tmW128,
                          const __grid_constant__ CUtensorMap tmW16,
@@ -121,6 +130,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int n_rounds = (n_tiles + TPR - 1) / TPR;
   const int n_k = p.H / BK;
 
+  // Programmatic dependent launch: the prologue below (barriers, TMEM) overlaps
+  // the previous kernel's tail; h and the workspace are touched only after
+  // grid_dep_wait.
+  grid_dep_launch();
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(full(s), 1);
@@ -133,27 +146,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&tmW128);
   }
   for (int i = threadIdx.x; i < 4 * Npad; i += THREADS) best[i] = 0ull;
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), tmem_cols);
     tmem_relinquish();
   }
+  grid_dep_wait();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto tile_rows = [&](int t) {
-    const int a = row0 + t * BM;
-    const int e = a + BM < row_end ? a + BM : row_end;
-    return e - a;
-  };
+  auto tile_rows = [&](int t) { return tile_rows_of(row0, row_end, t); };
 
 #define WAIT_OR(barrier, parity, on_fail) \
-  if (!mbar_wait_bounded((barrier), (parity), abort_flag, p.dev_status)) on_fail
+  if (!mbar_wait_bounded<kShortWait>((barrier), (parity), abort_flag, p.dev_status, p.wait_ns)) on_fail
 #define WARP_WAIT_OR(barrier, parity, on_fail) \
-  if (!mbar_wait_warp((barrier), (parity), abort_flag, p.dev_status)) on_fail
+  if (!mbar_wait_warp<kShortWait>((barrier), (parity), abort_flag, p.dev_status, p.wait_ns)) on_fail
 
   if (n_tiles > 0 && warp == 0 && lane == 0) {
     // ------------------------------------------------------------ producer
@@ -281,6 +292,8 @@ __global__ void __launch_bounds__(256) lmhead_reduce_kernel(const uint64_t* __re
                                                             int n_ctas, int Npad,
                                                             int32_t* __restrict__ argmax,
                                                             float* __restrict__ max_logit) {
+  grid_dep_launch();
+  grid_dep_wait();  // the candidate keys come from the main kernel
   const int r = blockIdx.x;
   uint64_t k = 0ull;
   for (int c = threadIdx.x; c < n_ctas; c += blockDim.x)
@@ -337,8 +350,10 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     rc = encode_tmap_bf16(&tw16, W, 2, dims, strides, box16);
     if (rc != ORTHRUS_OK) return rc;
   }
-  if (!opt_in_smem(reinterpret_cast<const void*>(lmh::lmhead_argmax_kernel), lmh::SMEM_LIMIT))
-    return ORTHRUS_ECUDA;
+  const uint64_t wait_ns = wait_limit_ns();
+  auto* kfn = wait_ns < kShortWaitNs ? lmh::lmhead_argmax_kernel<true>
+                                     : lmh::lmhead_argmax_kernel<false>;
+  if (!opt_in_smem(reinterpret_cast<const void*>(kfn), lmh::SMEM_LIMIT)) return ORTHRUS_ECUDA;
   const int grid = static_cast<int>((static_cast<long long>(V) + lmh::GROUP - 1) / lmh::GROUP <
                                             sms
                                         ? (V + lmh::GROUP - 1) / lmh::GROUP
@@ -357,6 +372,7 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     lmh::Params p;
     p.part_keys = keys;
     p.dev_status = dev_status;
+    p.wait_ns = wait_ns;
     p.R = Rp;
     p.Npad = pl.Npad;
     p.H = H;
@@ -364,11 +380,13 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     p.TPR = pl.TPR;
     p.NS = pl.NS;
     p.stage_bytes = pl.stage_bytes;
-    lmh::lmhead_argmax_kernel<<<grid, lmh::THREADS, pl.smem, s>>>(tw128, tw16, th, p);
-    if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
-    lmh::lmhead_reduce_kernel<<<Rp, 256, 0, s>>>(keys, grid, pl.Npad, argmax + r0,
-                                                 max_logit ? max_logit + r0 : nullptr);
-    if (cudaGetLastError() != cudaSuccess) return ORTHRUS_ECUDA;
+    rc = launch_kernel(kfn, dim3(grid), dim3(lmh::THREADS),
+                       static_cast<size_t>(pl.smem), s, tw128, tw16, th, p);
+    if (rc != ORTHRUS_OK) return rc;
+    rc = launch_kernel(lmh::lmhead_reduce_kernel, dim3(Rp), dim3(256), 0, s,
+                       static_cast<const uint64_t*>(keys), grid, pl.Npad, argmax + r0,
+                       max_logit ? max_logit + r0 : static_cast<float*>(nullptr));
+    if (rc != ORTHRUS_OK) return rc;
   }
   return ORTHRUS_OK;
 }
@@ -385,8 +403,9 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
 // per-CTA candidate keys in a fixed array in the library's own device memory
 // instead of a caller workspace.
 //
-//   * The array holds at most kNoAllocMaxCtas * 256 keys (512 KB).  It lives in
-//     every GPU that loads the library, for as long as the process runs.
+//   * The array holds kNoAllocMaxCtas * 256 candidate keys plus the 256-byte
+//     tail the workspace entry point asks for (512.25 KB).  It lives in every
+//     GPU that loads the library, for as long as the process runs.
 //   * All calls share it and it keeps the last call's contents.  Nothing in it
 //     needs to start at zero: every CTA overwrites all of its keys before the
 //     reduction reads them.  Calls whose kernels overlap on the GPU (other
@@ -402,7 +421,12 @@ namespace orthrus {
 namespace lmh {
 
 constexpr int kNoAllocMaxCtas = 256;
-static __device__ __align__(256) uint64_t g_noalloc_keys[kNoAllocMaxCtas * MAX_PASS_ROWS];
+// Exactly what orthrus_lmhead_workspace_size asks for on a kNoAllocMaxCtas-SM
+// device: kNoAllocMaxCtas * MAX_PASS_ROWS keys and 256 bytes more.
+static __device__ __align__(256) uint64_t g_noalloc_keys[kNoAllocMaxCtas * MAX_PASS_ROWS + 32];
+static_assert(sizeof(g_noalloc_keys) ==
+                  static_cast<size_t>(kNoAllocMaxCtas) * MAX_PASS_ROWS * sizeof(uint64_t) + 256,
+              "no-alloc scratch must cover the workspace size at the largest SM count");
 
 // Device address of g_noalloc_keys on the current device (looked up once per
 // device; the symbol's host-side name is only a handle, never a pointer the

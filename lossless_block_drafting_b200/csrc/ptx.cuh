@@ -52,6 +52,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait whose suspension (while the phase is incomplete) lasts at most
+// about `hint_ns` nanoseconds before it returns false.
+__device__ __forceinline__ bool mbar_try_wait_for(uint32_t bar, uint32_t parity,
+                                                  uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // ---------------------------------------------------------------- proxies
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA,
 // tcgen05.mma operand reads).
@@ -122,6 +136,19 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
   return p;
+}
+
+// ------------------------------------------ programmatic dependent launch
+// Lets the next kernel in the stream (launched with programmatic stream
+// serialisation) be scheduled once every CTA of this grid has issued it or
+// exited.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until every grid this one depends on has completed and its memory
+// operations are visible (returns at once when there is none).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05

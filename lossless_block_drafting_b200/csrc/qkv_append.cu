@@ -41,6 +41,8 @@ template <int D>
 __global__ void __launch_bounds__(THREADS) qkv_append_kernel(const Params p) {
   constexpr int E = D / 32;  // elements per lane
   __shared__ float2 cs[D / 2];
+  grid_dep_launch();
+  grid_dep_wait();  // qkv, ctx_lens and the cache may come from the previous kernel
   const int t = blockIdx.x;
   const int b = t / p.K, i = t - b * p.K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -140,8 +142,6 @@ extern "C" int orthrus_block_qkv_append(const void* qkv, const void* q_norm_w,
   const dim3 grid(static_cast<unsigned>(cache->B * K));
   const cudaStream_t s = as_stream(stream);
   if (cache->d == 128)
-    qkv::qkv_append_kernel<128><<<grid, qkv::THREADS, 0, s>>>(p);
-  else
-    qkv::qkv_append_kernel<64><<<grid, qkv::THREADS, 0, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? ORTHRUS_OK : ORTHRUS_ECUDA;
+    return launch_kernel(qkv::qkv_append_kernel<128>, grid, dim3(qkv::THREADS), 0, s, p);
+  return launch_kernel(qkv::qkv_append_kernel<64>, grid, dim3(qkv::THREADS), 0, s, p);
 }

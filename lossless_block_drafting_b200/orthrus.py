@@ -57,6 +57,7 @@ def load(path: str | None = None):
         sig = {
             "orthrus_status_str": ([I], ctypes.c_char_p),
             "orthrus_abi_version": ([], I),
+            "orthrus_set_wait_limit_ns": ([ctypes.c_uint64], I),
             "orthrus_block_attn_workspace_size": ([I, I, I, I, I, PSZ], I),
             "orthrus_block_attn": ([V, PC, I, I, I, V, V, SZ, V, V], I),
             "orthrus_lmhead_workspace_size": ([I, I, PSZ], I),
@@ -75,6 +76,11 @@ def load(path: str | None = None):
             f.restype = res
         _lib = lib
         return lib
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Limit after which a kernel's bounded waits give up (0 restores 2 s)."""
+    _check(load().orthrus_set_wait_limit_ns(int(ns)), "orthrus_set_wait_limit_ns")
 
 
 def status_str(status: int) -> str:

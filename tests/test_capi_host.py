@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     for want in ("orthrus_block_attn", "orthrus_lmhead_argmax", "orthrus_verify",
                  "orthrus_kv_commit", "orthrus_verify_commit", "orthrus_row_argmax_f32",
                  "orthrus_block_attn_workspace_size", "orthrus_lmhead_workspace_size",
-                 "orthrus_status_str", "orthrus_abi_version", "orthrus_block_qkv_append"):
+                 "orthrus_status_str", "orthrus_abi_version", "orthrus_block_qkv_append",
+                 "orthrus_set_wait_limit_ns"):
         assert want in names
 
 
@@ -44,7 +45,13 @@ def test_status_strings(lib):
         s = ob.status_str(code)
         assert s.startswith("ORTHRUS")
     assert "unknown" in ob.status_str(-99)
-    assert lib.orthrus_abi_version() == 1
+    assert lib.orthrus_abi_version() == 2
+
+
+def test_wait_limit_setter_accepts_any_value(lib):
+    # host-only: the limit is read at each launch; 0 restores the default
+    for ns in (1, 100, 2_000_000_000, 0):
+        assert lib.orthrus_set_wait_limit_ns(ns) == ob.OK
 
 
 def _view(B=1, Hkv=2, cap=64, d=64, k=0x1000, v=0x2000, lens=0x3000):

@@ -6,7 +6,8 @@ keeps its scratch in the library's own fixed device array.  This file is named
 to be collected last, so a failure here never hides another test's result.  It
 calls both entry points through the C ABI twice in a row (the scratch keeps
 the previous call's contents, which must not leak into the next result) and
-requires identical argmax and max-logit outputs.
+requires identical argmax and max-logit outputs.  R = 300 runs two passes of
+the kernel over the same scratch (rows 0..255, then 256..299).
 """
 import ctypes
 
@@ -24,7 +25,7 @@ def _c(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("R,H,V", [(32, 4096, 151936), (5, 256, 3000)])
+@pytest.mark.parametrize("R,H,V", [(32, 4096, 151936), (5, 256, 3000), (300, 256, 5000)])
 def test_noalloc_matches_workspace_entry_point_twice(R, H, V):
     libbuild.build()
     lib = ob.load()
