@@ -66,6 +66,12 @@ constexpr int TN = 64;        // keys per compute tile
 // the TMA engines near HBM bandwidth (measured: 64-row boxes top out at about
 // 80% of it, 128-row boxes near 97%).
 constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
+// Partial O layout: [ROWS / BR row blocks][slot][D / 4 column quads][BR rows][4]
+// floats.  A warp's store of one column quad for its 32 rows covers four whole
+// 128-byte lines, and since the pieces of a segment occupy consecutive slots,
+// one row block of all of them is one contiguous range: the merge fetches it
+// with a single bulk copy.
+constexpr int BR = 8;
 constexpr int THREADS = 384;  // 12 warps: TMA, MMA, TMEM alloc, spare, 2 softmax groups
 constexpr int TMEM_COLS = 512;
 // TMEM columns: two S buffers of 2 * TN fp32 columns, one per load group in
@@ -116,7 +122,7 @@ static_assert(RING > Layout<64>::NK + NSB + 1 && RING > Layout<128>::NK + NSB + 
 
 struct Params {
   const int32_t* ctx_lens;
-  float* part_o;      // [slots][ROWS][D] unnormalised O of each piece
+  float* part_o;      // [ROWS / 8][slots][D / 4][8][4] unnormalised O of each piece
   float2* part_ml;    // [slots][ROWS] (m in log2 units, l)
   unsigned long long* gbar;  // grid-barrier arrival ticket counter (starts at 0)
   unsigned long long* seg_cnt;  // [SMs] per-segment completion counters (start at 0)
@@ -125,6 +131,7 @@ struct Params {
   int32_t* dev_status;
   unsigned long long wait_ns;  // bounded-wait limit
   int B, K, Hq, Hkv, G, Gc, nhc, cap, mask_mode;
+  int slots;          // pieces the workspace holds (segments + grid size)
   int balance;        // per-segment partition: claim the tail groups dynamically
   float sl2;          // softmax scale * log2(e)
 };
@@ -538,7 +545,10 @@ __device__ void merge_rows(const Params& p, int P, long long r0, long long r1, i
         const long long c = base + k;
         const bool live = c <= sp.c1 && has_piece(c);
         ml[k] = live ? __ldcg(&p.part_ml[(s + c) * ROWS + r]) : make_float2(-INFINITY, 0.f);
-        const float* src = p.part_o + ((s + c) * ROWS + r) * D + lane * PER;
+        // partial O layout: [ROWS / BR][slot][D / 4 column quads][BR][4]
+        const float* src =
+            p.part_o + ((((r / BR) * static_cast<long long>(p.slots) + s + c) * (D / 4) +
+                         lane * PER / 4) * BR + r % BR) * 4 + (lane * PER) % 4;
         if constexpr (PER == 4) {
           const float4 t = live ? __ldcg(reinterpret_cast<const float4*>(src))
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -582,29 +592,32 @@ __device__ void merge_rows(const Params& p, int P, long long r0, long long r1, i
   }
 }
 
-// Per-segment partition: CTA k of the cn CTAs of segment s merges rows
-// [row0, row1) of that segment, RC rows per round.  Warp 0 bulk-copies the
-// rows' fp32 partial O of up to NPB pieces into shared memory (one contiguous
-// copy per piece, issued from all lanes, all in flight at once) while other
-// threads load the pieces' (m, l); then thread (row, float4 column) folds the
-// batch into its running (M, L, acc) -- every thread of a row derives the
-// same weights from the shared (m, l) table -- and finally writes acc / L as
-// bf16.  `buf` is the idle K/V ring (1024-aligned).
+// Per-segment partition: CTA k of the cn CTAs of segment s merges the row
+// blocks of [row0, row1) of that segment (row0 is a multiple of BR), one block
+// per round, the pieces in batches of up to NPB.  Lane 0 of warp 0 fetches the
+// block of every piece of the batch with ONE bulk copy (no multicast); at the
+// same time warp 1 + rr takes row rr: its lanes load the pieces' (m, l),
+// reduce the row's running maximum and normaliser with shuffles and store each
+// piece's weight.  Then thread (row, column quad) adds up its pieces' weighted
+// partials and writes its four output columns as bf16.  `buf` is the idle
+// K/V ring.
 template <int D, bool kShortWait>
-__device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int row1, int warp,
-                              int lane, uint8_t* buf, volatile int* abort_flag) {
-  constexpr int RC = 8;                                  // rows per round
-  constexpr int Q4 = D / 4;                              // float4 columns of a row
-  constexpr int PIECE = RC * D * 4;                      // bytes of one piece's rows
-  constexpr int HEAD = 4096;                             // barrier, (m, l) table
+__device__ void merge_segment(const Params& p, const OwnSeg own, int row0, int row1,
+                              uint8_t* buf, volatile int* abort_flag) {
+  constexpr int Q4 = D / 4;                 // float4 column quads of a row
+  constexpr int BLK = BR * D * 4;           // bytes of one row block of one piece
+  constexpr int HEAD = 4096;                // mbarrier, weights, scales
   constexpr int AVAIL = (Layout<D>::NK + Layout<D>::NV) * Layout<D>::KV_BYTES - HEAD;
-  // one (m, l) load per thread of warps 1.., one or two bulk copies per lane of warp 0
-  constexpr int NPB = AVAIL / PIECE < (THREADS - 32) / RC ? AVAIL / PIECE : (THREADS - 32) / RC;
-  static_assert(NPB >= 1 && NPB <= 64, "merge batch: 1..64 pieces (two per lane of warp 0)");
-  static_assert(64 + NPB * RC * 8 <= HEAD, "merge (m, l) table");
+  constexpr int NPB = AVAIL / BLK < 96 ? AVAIL / BLK : 96;  // pieces per batch
+  static_assert(NPB >= 32 && 64 + BR * NPB * 4 + 2 * BR * 4 <= HEAD && BR * Q4 <= THREADS &&
+                    (1 + BR) * 32 <= THREADS,
+                "merge staging");
   const uint32_t bar = smem_u32(buf);
-  float2* ml_s = reinterpret_cast<float2*>(buf + 64);                         // [NPB][RC]
-  const float4* o_s = reinterpret_cast<const float4*>(buf + HEAD);            // [NPB][RC][Q4]
+  float* wt = reinterpret_cast<float*>(buf + 64);             // [BR][NPB] piece weights
+  float* rs = wt + BR * NPB;                                  // [BR] rescale of the running sum
+  float* rinv = rs + BR;                                      // [BR] 1 / normaliser
+  const float4* o_s = reinterpret_cast<const float4*>(buf + HEAD);  // [NPB][Q4][BR]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
@@ -621,79 +634,88 @@ __device__ void merge_segment(const Params& p, const OwnSeg& own, int row0, int 
     return dense || mul_div(j, own.ns, own.cn) != mul_div(j + 1, own.ns, own.cn);
   };
   const int nseg = p.Hkv * p.nhc;
-  const int b = static_cast<int>(own.s / nseg), seg = static_cast<int>(own.s % nseg);
-  const int g = seg / p.nhc, hc = seg % p.nhc;
-  const int tr = threadIdx.x / Q4, tq = threadIdx.x % Q4;  // this thread's (row, float4)
+  const int s_own = static_cast<int>(own.s);  // < grid size
+  const int b = s_own / nseg, seg = s_own - b * nseg;
+  const int g = seg / p.nhc, hc = seg - g * p.nhc;
+  const int tr = threadIdx.x % BR, tq = threadIdx.x / BR;  // this thread's (row, quad)
+  const int rr = warp - 1;                                  // the row of warps 1..BR
+  const long long slot0 = own.s + own.c0;
   uint32_t phase = 0;
-  for (int rb = row0; rb < row1; rb += RC) {
-    const int nr = row1 - rb < RC ? row1 - rb : RC;
+  for (int rb = row0; rb < row1; rb += BR) {
+    const int row = rb + tr;
+    const bool on = tq < Q4 && row < row1;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float M = -INFINITY, L = 0.f;
+    float M = -INFINITY, L = 0.f;  // running (max, normaliser) of row rb + rr (warps 1..BR)
     for (int j0 = 0; j0 < own.cn; j0 += NPB) {
       const int nb = own.cn - j0 < NPB ? own.cn - j0 : NPB;
-      if (warp == 0) {
-        // Lane l copies pieces l and l + 32 of the batch (issue is parallel:
-        // one bulk copy costs ~150 cycles of issue in a single thread).
-        const bool on0 = lane < nb && live(j0 + lane);
-        const bool on1 = lane + 32 < nb && live(j0 + lane + 32);
-        const uint32_t n_on = __popc(__ballot_sync(0xFFFFFFFFu, on0)) +
-                              __popc(__ballot_sync(0xFFFFFFFFu, on1));
-        if (lane == 0) mbar_arrive_expect_tx(bar, n_on * nr * D * 4);
-        __syncwarp();
-        if (on0 || on1) fence_proxy_async_global();  // partials were written by generic stores
+      if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(bar, nb * BLK);
+        fence_proxy_async_global();  // the partials were written by generic stores
+        bulk_load(bar + HEAD,
+                  p.part_o + (static_cast<long long>(rb / BR) * p.slots + slot0 + j0) * (BLK / 4),
+                  nb * BLK, bar);
+      } else if (rr >= 0 && rr < BR) {
+        // lane l holds pieces l, l + 32, ... of the batch (all loads in flight)
+        constexpr int PL = (NPB + 31) / 32;
+        const bool row_on = rb + rr < row1;
+        float2 mlr[PL];
+        float mb = M;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (!(u == 0 ? on0 : on1)) continue;
-          const int jj = lane + 32 * u;
-          const long long slot = own.s + own.c0 + j0 + jj;
-          bulk_load(smem_u32(buf + HEAD + jj * PIECE), p.part_o + (slot * ROWS + rb) * D,
-                    nr * D * 4, bar);
+        for (int u = 0; u < PL; ++u) {
+          const int j = lane + 32 * u;
+          mlr[u] = (j < nb && row_on && live(j0 + j))
+                       ? __ldcg(p.part_ml + (slot0 + j0 + j) * ROWS + rb + rr)
+                       : make_float2(-INFINITY, 0.f);
+          mb = fmaxf(mb, mlr[u].x);
         }
-      } else if (threadIdx.x - 32 < nb * RC) {
-        const int t = threadIdx.x - 32;
-        const int jj = t / RC, r = t % RC;
-        const long long slot = own.s + own.c0 + j0 + jj;
-        ml_s[t] = (r < nr && live(j0 + jj)) ? __ldcg(p.part_ml + slot * ROWS + rb + r)
-                                            : make_float2(-INFINITY, 0.f);
+        for (int o = 16; o > 0; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, o));
+        float lsum = 0.f;
+#pragma unroll
+        for (int u = 0; u < PL; ++u) {
+          const int j = lane + 32 * u;
+          // empty or dead pieces weigh 0 (their partial O is never read)
+          const float w = mlr[u].x == -INFINITY ? 0.f : fast_exp2(mlr[u].x - mb);
+          if (j < nb) wt[rr * NPB + j] = w;
+          lsum += w * mlr[u].y;
+        }
+        for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xFFFFFFFFu, lsum, o);
+        const float sc = (M == -INFINITY || mb == -INFINITY) ? 0.f : fast_exp2(M - mb);
+        L = L * sc + lsum;
+        M = mb;
+        if (lane == 0) {
+          rs[rr] = sc;
+          rinv[rr] = L > 0.f ? 1.f / L : 0.f;
+        }
       }
-      // A wait that gives up still lets this round's copies land before the
-      // CTA leaves (they target its shared memory); then every thread returns.
+      // A wait that gives up still lets the copy land before the CTA leaves
+      // (it targets this CTA's shared memory); then every thread returns.
       if (!mbar_wait_bounded<kShortWait>(bar, phase, abort_flag, p.dev_status, p.wait_ns))
         mbar_wait_drain(bar, phase, p.dev_status);
       phase ^= 1u;
       __syncthreads();
       if (*abort_flag) return;  // read by all threads between the same two barriers
-      if (tr < nr) {
-        float mb = M;
-        for (int jj = 0; jj < nb; ++jj) mb = fmaxf(mb, ml_s[jj * RC + tr].x);
-        if (mb != -INFINITY) {
-          const float sc = M == -INFINITY ? 0.f : fast_exp2(M - mb);
-          acc.x *= sc;
-          acc.y *= sc;
-          acc.z *= sc;
-          acc.w *= sc;
-          L *= sc;
-          M = mb;
-          for (int jj = 0; jj < nb; ++jj) {
-            const float2 ml = ml_s[jj * RC + tr];
-            if (ml.x == -INFINITY) continue;  // dead or empty piece: its O may be stale
-            const float wj = fast_exp2(ml.x - M);
-            const float4 x = o_s[(jj * RC + tr) * Q4 + tq];
-            L += wj * ml.y;
-            acc.x += wj * x.x;
-            acc.y += wj * x.y;
-            acc.z += wj * x.z;
-            acc.w += wj * x.w;
-          }
+      if (on) {
+        const float sc = rs[tr];
+        acc.x *= sc;
+        acc.y *= sc;
+        acc.z *= sc;
+        acc.w *= sc;
+        for (int jj = 0; jj < nb; ++jj) {
+          const float w = wt[tr * NPB + jj];
+          if (w == 0.f) continue;  // empty or dead piece: its partial may be stale
+          const float4 x = o_s[(jj * Q4 + tq) * BR + tr];
+          acc.x += w * x.x;
+          acc.y += w * x.y;
+          acc.z += w * x.z;
+          acc.w += w * x.w;
         }
       }
       __syncthreads();
     }
-    if (tr < nr) {
-      const int row = rb + tr;
+    if (on) {
       const int i = row / p.Gc, hh = row % p.Gc;
       if (hc * p.Gc + hh < p.G) {
-        const float inv = L > 0.f ? 1.f / L : 0.f;
+        const float inv = rinv[tr];
         const int h = g * p.G + hc * p.Gc + hh;
         __nv_bfloat16* dst =
             p.out + ((static_cast<long long>(b) * p.K + i) * p.Hq + h) * D + tq * 4;
@@ -750,24 +772,23 @@ __global__ void __launch_bounds__(THREADS, 1)
   float2* ml_xchg = reinterpret_cast<float2*>(smem + Ly::OFF_ML);
 
   // Programmatic dependent launch: the next kernel in the stream may be
-  // scheduled now (its CTAs land on SMs as this grid's CTAs exit).  Until
-  // grid_dep_wait below this kernel touches only its own shared and tensor
-  // memory, L2 prefetches and ctx_lens, which it reads speculatively (through
-  // L2, never L1) and reads again after the wait.
+  // scheduled now; its CTAs land on SMs as this grid's CTAs exit (one CTA
+  // fills an SM's shared memory).  Everything a preceding kernel may write
+  // (ctx_lens, q, the cache, the workspace, dev_status) is touched only after
+  // grid_dep_wait.
   grid_dep_launch();
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK2);
+    prefetch_tmap(&tmK1);
+  } else if (threadIdx.x == 64) {
+    prefetch_tmap(&tmV2);
+    prefetch_tmap(&tmV1);
+  }
 
   // The CTA's tile range and its starting cursor are computed by warp 0 and
-  // shared.  With up to 32 sequences a speculative schedule from the lengths
-  // as they stand is computed before the dependency wait and kept if the
-  // lengths read after the wait are the same.
+  // shared, while warp 1 initialises the barriers.
   long long* sched = reinterpret_cast<long long*>(smem + Ly::OFF_SCHED);
-  const bool spec = p.B <= 32;
-  int spec_raw = 0;
-  if (warp == 0 && spec) {
-    spec_raw = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
-    warp_schedule_small(p, gridDim.x, blockIdx.x, lane, false, sched, spec_raw);
-    __syncwarp();
-  }
 
   const int nseg = p.Hkv * p.nhc;
   // Per-segment partition: this CTA's segment (s = -1 in stream-K mode),
@@ -800,7 +821,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   OwnSeg pr_own{-1, 0, 0, 0, 0};
   Cursor pr_c{};
   int pr_n = 0, pr_j = 0, pr_cur = -2;
-  int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0;
+  int pr_sg = 0, pr_sg_end = 0, pr_pool0 = 0, pr_ngr = 0, pr_gclaims = 0, pr_tile0 = 0;
   bool pr_grabbing = false, pr_dry = true;
   unsigned long long pr_pend = 0;
   const uint64_t pr_policy = policy_evict_first();
@@ -823,7 +844,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_arrive(item_full(slot));
     if (flags & kItemNone) return true;
     if (flags & kItemPieceFirst) {
-      if (!mbar_wait_bounded<kShortWait>(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status, p.wait_ns))
+      if (!mbar_try_wait(q_empty, (pr_pieces & 1) ^ 1) &&
+          !mbar_wait_bounded<kShortWait>(q_empty, (pr_pieces & 1) ^ 1, abort_flag, p.dev_status,
+                                         p.wait_ns))
         return false;
       mbar_arrive_expect_tx(q_full, static_cast<uint32_t>(p.Gc * p.K * D * 2));
       for (int c = 0; c < Ly::CHUNKS; ++c)
@@ -832,8 +855,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const bool pair = flags & kItemPair;
     const int stage = pr_gi % NK;
-    if (!mbar_wait_bounded<kShortWait>(empty_k(stage), ((pr_gi / NK) & 1) ^ 1, abort_flag, p.dev_status,
-                           p.wait_ns))
+    if (!mbar_try_wait(empty_k(stage), ((pr_gi / NK) & 1) ^ 1) &&
+        !mbar_wait_bounded<kShortWait>(empty_k(stage), ((pr_gi / NK) & 1) ^ 1, abort_flag,
+                                       p.dev_status, p.wait_ns))
       return false;
     mbar_arrive_expect_tx(full_k(stage), (pair ? 2 : 1) * Ly::HALF * Ly::CHUNKS);
     for (int c = 0; c < Ly::CHUNKS; ++c)
@@ -853,36 +877,48 @@ __global__ void __launch_bounds__(THREADS, 1)
     pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);
     pr_grabbing = true;
   };
-  auto next_group = [&]() -> int {
+  // Work units are (first tile << 1) | pair.  The static run and the pool's
+  // first claims are 128-key groups; the pool's last groups (one per sibling)
+  // are handed out as single 64-key tiles, which halves the spread of the
+  // siblings' finishing times.
+  auto group_unit = [&](int g) { return (4 * g) | (2 * g + 1 < pr_own.ns ? 1 : 0); };
+  auto next_unit = [&]() -> int {
     if (pr_sg < pr_sg_end) {
       const int g = pr_sg++;
       if (!pr_grabbing && !pr_dry && pr_sg_end - pr_sg <= 1) start_claims();
-      return g;
+      return group_unit(g);
     }
     if (pr_dry) return -1;
     if (!pr_grabbing) start_claims();
-    const long long g = pr_pool0 + static_cast<long long>(pr_pend);
-    if (g >= pr_ngr) {
-      pr_dry = true;
-      return -1;
+    const long long c = static_cast<long long>(pr_pend);
+    int u;
+    if (c < pr_gclaims) {
+      u = group_unit(pr_pool0 + static_cast<int>(c));
+    } else {
+      const long long t = pr_tile0 + (c - pr_gclaims);
+      if (t >= pr_own.ns) {
+        pr_dry = true;
+        return -1;
+      }
+      u = static_cast<int>(t) << 1;
     }
     pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);  // next claim, in flight
-    return static_cast<int>(g);
+    return u;
   };
   // Before the barrier (pre) no other role runs yet, so only groups that need
   // no wait are emitted: the first NK (fresh K stages) of the first piece.
   auto produce = [&](int limit, bool pre) {
     if (pr_own.s >= 0 && p.balance) {
       if (pr_cur == -2) {
-        pr_cur = next_group();
+        pr_cur = next_unit();
         if (pr_cur < 0) emit(0, pr_own.L, static_cast<int>(pr_own.s), kItemNone);
       }
       while (pr_cur >= 0 && pr_gi < limit) {
-        const int nxt = next_group();
-        const bool pair = 2 * pr_cur + 1 < pr_own.ns;
+        const int nxt = next_unit();
+        const bool pair = pr_cur & 1;
         const int flags = (pair ? kItemPair : 0) | (pr_gi == 0 ? kItemPieceFirst : 0) |
                           (nxt < 0 ? (kItemPieceLast | kItemEnd) : 0);
-        if (!emit(2 * pr_cur, pr_own.L, static_cast<int>(pr_own.s), flags)) {
+        if (!emit(pr_cur >> 1, pr_own.L, static_cast<int>(pr_own.s), flags)) {
           pr_cur = -1;
           break;
         }
@@ -913,7 +949,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   };
 
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 32) {
     for (int s = 0; s < NK; ++s) {
       mbar_init(full_k(s), 1);
       mbar_init(empty_k(s), 1);
@@ -938,30 +974,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; i < RING; ++i) mbar_init(item_full(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
-    if (spec) {
-      // Warm L2 with the first groups of the speculative schedule while the
-      // previous kernel finishes (a stale schedule only wastes the prefetch).
-      prefetch_tmap(&tmK2);
-      prefetch_tmap(&tmV2);
-      const OwnSeg o = read_own();
-      if (o.s >= 0) {
-        const int b = static_cast<int>(o.s / nseg), seg = static_cast<int>(o.s % nseg);
-        const int kvbase = (b * p.Hkv + seg / p.nhc) * p.cap;
-        int t0 = static_cast<int>(sched[4] >> 32), t1 = t0 + static_cast<int>(sched[1] - sched[0]);
-        if (p.balance) {
-          const int ngr = (o.ns + 1) / 2;
-          const int fs = static_cast<int>(mul_div(3 * ngr, 1, 4 * o.cn));
-          t0 = 2 * (static_cast<int>(blockIdx.x) - o.c0) * fs;
-          t1 = t0 + 2 * fs;
-        }
-        if (t1 > t0 + 2 * NK) t1 = t0 + 2 * NK;
-        for (int t = t0; t < t1; t += 2)
-          for (int c = 0; c < Ly::CHUNKS; ++c) {
-            tma_prefetch_2d(&tmK2, c * 64, kvbase + t * TN);
-            tma_prefetch_2d(&tmV2, c * 64, kvbase + t * TN);
-          }
-      }
-    }
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -981,23 +993,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_proxy_async_smem();
   }
 
-  // Everything a preceding kernel may write (ctx_lens, q, the cache, the
-  // workspace, dev_status) is read or written only after this point.
   grid_dep_wait();
   if (warp == 0) {
-    if (spec) {
-      const int raw = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
-      if (!__all_sync(0xFFFFFFFFu, raw == spec_raw))
-        warp_schedule_small(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched, raw);
-      else if (blockIdx.x == 0 && lane < p.B && (raw < 0 || raw > p.cap - p.K))
-        report(p.dev_status, ORTHRUS_ECAPACITY);
-    } else {
-      warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
-    }
+    warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
     __syncwarp();
   }
+  // warps 0 and 1 meet: the barriers are initialised and the schedule written
+  if (warp < 2) asm volatile("bar.sync 2, 64;" ::: "memory");
   if (threadIdx.x == 0) {
-    // warp 0 wrote the schedule (the warp converged after it)
     pr_own = read_own();
     pr_c = read_start();
     pr_n = static_cast<int>(sched[1] - sched[0]);
@@ -1009,6 +1012,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       pr_sg = k * fs;
       pr_sg_end = pr_sg + fs;
       pr_dry = pr_pool0 >= pr_ngr;
+      const int pool = pr_ngr - pr_pool0;             // groups left to claim
+      pr_gclaims = pool > pr_own.cn ? pool - pr_own.cn : 0;
+      pr_tile0 = 2 * (pr_pool0 + pr_gclaims);         // then tiles from here
     }
     produce(NK, true);
   }
@@ -1032,8 +1038,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (pr_pieces > 0) mbar_wait_drain(q_full, (pr_pieces - 1) & 1, p.dev_status);
   } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------- V producer
-    prefetch_tmap(&tmV2);
-    prefetch_tmap(&tmV1);
     const uint64_t policy = policy_evict_first();
     int gi = 0;
     for (;;) {
@@ -1112,7 +1116,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // = two 8-row swizzle atoms (2048 B); d chunks Ly::KV_CHUNK apart.
       vd[kk] = make_sdesc(sb0 + Ly::OFF_V + kk * 2048, Ly::KV_CHUNK, 1024, kSwizzle128B);
     int pieces_done = 0, jp = 0, gi = 0, j = 0;
-    int pf_uses[2 * NSB] = {0, 0, 0, 0};  // completed phases seen per P barrier
+    uint32_t pf_par = 0;  // bit pb: parity of P barrier pb's next phase (kept in a register)
     bool fail = false;
     for (;;) {
       const int slot = gi % RING;
@@ -1130,8 +1134,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int h = 0; h < ntl; ++h, ++j) {
         const int w = j & 1;
         const int pb = 2 * gb + h;
-        WAIT_OR(p_full(pb), pf_uses[pb] & 1, { fail = true; break; });
-        ++pf_uses[pb];
+        WAIT_OR(p_full(pb), (pf_par >> pb) & 1u, { fail = true; break; });
+        pf_par ^= 1u << pb;
         if (h == 0) {
           WAIT_OR(full_v(stage), (gi / NV) & 1, { fail = true; break; });
         }
@@ -1369,7 +1373,11 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (lane == 0) mbar_arrive(xchg_scale);
         }
         if (!idle_warp) {  // rows of all-padding warps are never merged
-          float* dst = p.part_o + (pslot * ROWS + r) * D;
+          // partial O in row blocks (BR rows x D / 4 quads x 4 floats): the
+          // warp's 32 rows of one column quad fill four whole lines
+          float4* dst = reinterpret_cast<float4*>(p.part_o) +
+                        ((r / BR) * static_cast<long long>(p.slots) + pslot) * (D / 4) * BR +
+                        r % BR;
 #pragma unroll
           for (int c0 = w * (D / 2); c0 < (w + 1) * (D / 2); c0 += 32) {
             uint32_t o0[32], o1r[32];
@@ -1387,7 +1395,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 2]) : 0.f);
               v.w = (a0 != 0.f ? a0 * __uint_as_float(o0[k + 3]) : 0.f) +
                     (a1 != 0.f ? a1 * __uint_as_float(o1r[k + 3]) : 0.f);
-              *reinterpret_cast<float4*>(dst + c0 + k) = v;
+              dst[((c0 + k) / 4) * BR] = v;
             }
           }
         }
@@ -1422,9 +1430,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     // siblings have added only after their last claim, so once the target is
     // reached the last CTA of the segment (which always has rows to merge)
     // puts the claim counter back to 0 for the next call.
+    // shares of whole BR-row blocks (the last CTA's share is never empty)
     const int k = static_cast<int>(blockIdx.x) - own.c0;
-    const int row0 = static_cast<int>(mul_div(k, RV, own.cn));
-    const int row1 = static_cast<int>(mul_div(k + 1, RV, own.cn));
+    const int nblk = (RV + BR - 1) / BR;
+    const int row0 = BR * static_cast<int>(mul_div(k, nblk, own.cn));
+    const int row1e = BR * static_cast<int>(mul_div(k + 1, nblk, own.cn));
+    const int row1 = row1e < RV ? row1e : RV;
     if (threadIdx.x == 0) {
       __threadfence();
       const unsigned long long add = k == 0 ? (1ull << 20) - (own.cn - 1) : 1ull;
@@ -1435,7 +1446,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         *reinterpret_cast<volatile unsigned long long*>(p.seg_next + own.s) = 0ull;
     }
     __syncthreads();
-    merge_segment<D, kShortWait>(p, own, row0, row1, warp, lane, smem + Ly::OFF_K, abort_flag);
+    merge_segment<D, kShortWait>(p, own, row0, row1, smem + Ly::OFF_K, abort_flag);
     return;
   }
 
@@ -1549,6 +1560,7 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   p.G = sh.G;
   p.Gc = sh.Gc;
   p.nhc = sh.nhc;
+  p.slots = static_cast<int>(slots);
   p.cap = cache->cap;
   p.mask_mode = mask_mode & 1;
   p.balance = (mask_mode & ORTHRUS_ATTN_DETERMINISTIC) ? 0 : 1;

@@ -25,8 +25,10 @@ void resolve_encode() {
 }
 }  // namespace
 
-int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                     const uint64_t* strides_bytes, const uint32_t* box) {
+namespace {
+int encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, CUtensorMapSwizzle swizzle,
+                const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                const uint32_t* box) {
   std::call_once(g_encode_once, resolve_encode);
   if (g_encode == nullptr) return ORTHRUS_ECUDA;
   cuuint64_t gdim[5];
@@ -39,11 +41,23 @@ int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_
     estride[i] = 1;
     if (i + 1 < rank) gstride[i] = strides_bytes[i];
   }
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
-                        const_cast<void*>(base), gdim, gstride, bdim, estride,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gdim,
+                        gstride, bdim, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ORTHRUS_OK : ORTHRUS_EINVAL;
+}
+}  // namespace
+
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, base, rank,
+                     dims, strides_bytes, box);
+}
+
+int encode_tmap_f32_plain(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tmap(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_NONE, base, rank,
+                     dims, strides_bytes, box);
 }
 
 bool opt_in_smem(const void* kernel, int bytes) {

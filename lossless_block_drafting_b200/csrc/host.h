@@ -18,6 +18,10 @@ namespace orthrus {
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box);
 
+// fp32 tiled tensor map without swizzle (same conventions as above).
+int encode_tmap_f32_plain(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                          const uint64_t* strides_bytes, const uint32_t* box);
+
 // Number of SMs of the current device (ORTHRUS_ECUDA on failure).
 int current_sm_count(int* sms);
 

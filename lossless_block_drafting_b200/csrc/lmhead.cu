@@ -11,10 +11,11 @@
 // dimension (h, K-major, N padded to a multiple of 32), fp32 accumulators in
 // TMEM.  Each CTA of a one-per-SM grid owns an equal, 16-row-granular slice of
 // the vocabulary; it streams W through a TMA ring (64 hidden elements = one
-// 128-byte swizzled row per stage, evict-first L2 policy) and keeps up to four
-// tiles' accumulators live at once so each h chunk is fetched once per four
-// W tiles.  Accumulators are double-buffered so the epilogue of one round
-// overlaps the MMAs of the next.  The epilogue (one thread per vocab row) maps
+// 128-byte swizzled row per stage, evict-first L2 policy) and keeps two to
+// four tiles' accumulators live at once so each h chunk is fetched once per
+// two to four W tiles.  While two rounds fit in TMEM (N <= 128) the
+// accumulators are double-buffered so the epilogue of one round overlaps the
+// MMAs of the next.  The epilogue (one thread per vocab row) maps
 // each logit to a 64-bit key (order-preserving value bits | inverted index,
 // so ties go to the smallest index), reduces across the warp with a
 // transposing butterfly, and keeps a per-warp best per column in shared
@@ -42,17 +43,25 @@ struct Params {
   uint64_t* part_keys;  // [gridDim.x][Npad]
   int32_t* dev_status;
   unsigned long long wait_ns;  // bounded-wait limit
-  int R, Npad, H, V, TPR, NS, stage_bytes;
+  int R, Npad, H, V, TPR, NB, NS, stage_bytes;
 };
 
 struct Plan {
-  int Npad, TPR, NS, stage_bytes, smem;
+  int Npad, TPR, NB, NS, stage_bytes, smem;
 };
 
+// Tiles per round TPR: every h chunk staged feeds TPR W tiles, so the
+// shared-memory fill per MMA shrinks as TPR grows (at N = 256 one tile per
+// stage would need about 96 B/clk per SM, two tiles 64 B/clk).  The round's
+// accumulators are double-buffered (NB = 2) while 2 * TPR * Npad fits the 512
+// TMEM columns; otherwise (Npad > 128) a single buffer holds two tiles and
+// the MMAs of the next round wait for the epilogue.
 inline Plan make_plan(int R) {
   Plan pl;
   pl.Npad = ((R + 31) / 32) * 32;
-  pl.TPR = MAX_PASS_ROWS / pl.Npad < 4 ? MAX_PASS_ROWS / pl.Npad : 4;
+  const int tpr = MAX_PASS_ROWS / pl.Npad;
+  pl.TPR = tpr < 2 ? 2 : (tpr > 4 ? 4 : tpr);
+  pl.NB = 2 * pl.TPR * pl.Npad <= 512 ? 2 : 1;
   pl.stage_bytes = pl.TPR * W_TILE_BYTES + pl.Npad * 128;
   const int fixed = 1024 /*align*/ + 4 * pl.Npad * 8 /*bests*/ + 64 * 8 /*barriers*/ + 16;
   pl.NS = (SMEM_LIMIT - fixed) / pl.stage_bytes;
@@ -117,7 +126,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* best = reinterpret_cast<uint64_t*>(smem + off_best);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + off_bar + 8 * (2 * NS + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const uint32_t tmem_cols = (2 * TPR * Npad) <= 256 ? 256u : 512u;
+  const int NB = p.NB;
+  const uint32_t tmem_cols = (NB * TPR * Npad) <= 256 ? 256u : 512u;
 
   // This CTA's vocabulary slice, in 16-row groups.
   const long long NG = (p.V + GROUP - 1) / GROUP;
@@ -209,10 +219,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     int it = 0;
     bool ok = true;
     for (int q = 0; ok && q < n_rounds; ++q) {
-      const int buf = q & 1;
+      const int buf = q % NB;
       const int ntr = n_tiles - q * TPR < TPR ? n_tiles - q * TPR : TPR;
-      if (q >= 2) {
-        WAIT_OR(acc_free(buf), ((q - 2) >> 1) & 1, break);
+      if (q >= NB) {
+        WAIT_OR(acc_free(buf), ((q - NB) / NB) & 1, break);
       }
       tc_fence_after();
       const uint32_t acc = tmem + static_cast<uint32_t>(buf * TPR * Npad);
@@ -243,9 +253,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint64_t* my_best = best + quarter * Npad;
     for (int q = 0; q < n_rounds; ++q) {
-      const int buf = q & 1;
+      const int buf = q % NB;
       const int ntr = n_tiles - q * TPR < TPR ? n_tiles - q * TPR : TPR;
-      WARP_WAIT_OR(acc_full(buf), (q >> 1) & 1, break);
+      WARP_WAIT_OR(acc_full(buf), (q / NB) & 1, break);
       tc_fence_after();
       for (int u = 0; u < ntr; ++u) {
         const int t = q * TPR + u;
@@ -378,6 +388,7 @@ extern "C" int orthrus_lmhead_argmax(const void* h, const void* W, int R, int H,
     p.H = H;
     p.V = V;
     p.TPR = pl.TPR;
+    p.NB = pl.NB;
     p.NS = pl.NS;
     p.stage_bytes = pl.stage_bytes;
     rc = launch_kernel(kfn, dim3(grid), dim3(lmh::THREADS),
