@@ -12,7 +12,12 @@ phase boundaries, so the attention launches' average duration is measured on
 the launching stream inside the timed region.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
-                    [--ctx L] [--block K] [--layers N] [--sweep]
+                    [--ctx L] [--block K] [--layers N] [--no-extras]
+
+On one GPU the line also carries, unless --no-extras: the ragged-batch step (8
+sequences, lengths U[1024, 32768], K 32, planted accept lengths U{0..32}; its
+LM head has R = 256 rows) and the verify-step sweep over K in {1,4,8,16,32} x
+context in {1024, 8192, 40960, 131072} (K = 1 is plain decoding).
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (the reference arm of this benchmark).  Under torchrun (N > 1) every
@@ -54,8 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--accept", type=int, default=4,
                     help="planted accepted length per step (drafts agree with the AR "
                          "argmax on this many leading rows)")
-    ap.add_argument("--sweep", action="store_true",
-                    help="also time K in {1,4,8,16,32} x L in {1024,8192,40960,131072}")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the ragged-batch step and the K x context sweep that a "
+                         "single-GPU run reports beside the headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--json-out", default=None)
@@ -205,17 +211,25 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- workload
 class Workload:
-    """Resident synthetic inputs for one replica of the decode step."""
+    """Resident synthetic inputs for one replica of the decode step.
 
-    def __init__(self, B, K, L, layers, accept, steps_total, device, seed=0):
+    lens: committed context length per sequence (an int gives every sequence
+    the same); accepts: planted accept length per sequence (the diffusion view's
+    final hidden states equal the AR view's on that many leading rows of the
+    block, so the drafts match the AR argmax there and nowhere else).  kv:
+    optional (k, v) lists of per-layer caches to share with another workload.
+    """
+
+    def __init__(self, B, K, lens, layers, accepts, steps_total, device, seed=0, kv=None):
         import torch
         from lossless_block_drafting_b200 import orthrus as ob
         self.ob = ob
-        self.B, self.K, self.L0, self.layers = B, K, L, layers
+        lens = [int(lens)] * B if isinstance(lens, int) else [int(x) for x in lens]
+        accepts = [int(accepts)] * B if isinstance(accepts, int) else [int(x) for x in accepts]
+        self.B, self.K, self.lens, self.layers = B, K, lens, layers
+        self.L0 = lens[0]
         Hq, Hkv, d, H, V = QWEN["Hq"], QWEN["Hkv"], QWEN["d"], QWEN["H"], QWEN["V"]
         self.Hq, self.Hkv, self.d, self.H, self.V = Hq, Hkv, d, H, V
-        # room for the committed length to grow by up to K per step
-        self.cap = L + K * (steps_total + 2)
         g = torch.Generator(device=device).manual_seed(seed)
         bf = torch.bfloat16
 
@@ -223,8 +237,14 @@ class Workload:
             x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
             return (x * std).to(bf) if std != 1.0 else x.to(bf)
 
-        self.k = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
-        self.v = [randn(B, Hkv, self.cap, d) for _ in range(layers)]
+        if kv is None:
+            # room for the committed length to grow by up to K per step
+            cap = max(lens) + K * (steps_total + 2)
+            self.k = [randn(B, Hkv, cap, d) for _ in range(layers)]
+            self.v = [randn(B, Hkv, cap, d) for _ in range(layers)]
+        else:
+            self.k, self.v = kv
+        self.cap = self.k[0].shape[2]
         # A step's inputs (both views' queries for every layer, both views' final
         # hidden states) live in one flat buffer, so one host->device copy
         # delivers them all in the end-to-end measurement.
@@ -242,17 +262,17 @@ class Workload:
         self.q_ar = [place(randn(B, K, Hq, d)) for _ in range(layers)]
         self.W = randn(V, H, std=0.02)
         self.h_ar = place(randn(B * K, H))
-        # the diffusion view's final states agree with the AR view's on the first
-        # `accept` rows of every block, so drafts match the AR argmax there
         self.h_diff = place(randn(B * K, H))
-        a = max(0, min(accept, K))
-        hv = self.h_diff.view(B, K, H)
-        hv[:, :a] = self.h_ar.view(B, K, H)[:, :a]
-        self.accept = a
-        self.ctx_lens = torch.full((B,), L, dtype=torch.int32, device=device)
+        hv, ha = self.h_diff.view(B, K, H), self.h_ar.view(B, K, H)
+        self.accepts = [max(0, min(a, K)) for a in accepts]
+        for b_, a in enumerate(self.accepts):
+            hv[b_, :a] = ha[b_, :a]
+        self.accept = self.accepts[0]
+        self.ctx_lens = torch.tensor(lens, dtype=torch.int32, device=device)
         self.ctx_init = self.ctx_lens.clone()
         self.attn_out = torch.empty(B, K, Hq, d, dtype=bf, device=device)
-        self.ws_attn = torch.zeros(ob.block_attn_workspace_size(B, Hq, Hkv, d, K), dtype=torch.uint8, device=device)
+        self.ws_attn = torch.zeros(ob.block_attn_workspace_size(B, Hq, Hkv, d, K),
+                                   dtype=torch.uint8, device=device)
         self.ws_lm = torch.empty(ob.lmhead_workspace_size(B * K, V), dtype=torch.uint8,
                                  device=device)
         self.draft = torch.empty(B * K, dtype=torch.int32, device=device)
@@ -268,29 +288,41 @@ class Workload:
     def launches_per_step(self):
         return 2 * self.layers + 2 * 2 + 1
 
+    def emitted_per_step(self):
+        """Tokens a step emits: the accepted drafts plus the correction (or the
+        last draft when all K are accepted), per sequence."""
+        return sum(min(a + 1, self.K) for a in self.accepts)
+
     def attn_bytes(self):
-        """Algorithmic bytes of one attention call at the starting context."""
-        kv = 2 * self.B * self.Hkv * self.d * 2 * (self.L0 + self.K)
+        """Algorithmic bytes of one attention call at the starting contexts:
+        K and V of every key each (sequence, KV head) reads, plus Q and O."""
+        kv = 2 * self.Hkv * self.d * 2 * sum(L + self.K for L in self.lens)
         qo = 2 * self.B * self.K * self.Hq * self.d * 2
         return kv + qo
 
     def lm_bytes(self):
         return self.V * self.H * 2 + self.B * self.K * self.H * 2
 
-    def step(self, stream, events=None):
-        """Issue one decode step on `stream`; events (if given) mark phase boundaries."""
+    def lm_flops(self):
+        return 2.0 * self.B * self.K * self.H * self.V
+
+    def step(self, stream, events=None, verify_only=False):
+        """Issue one decode step on `stream`; events (if given) mark phase
+        boundaries.  verify_only: the AR pass, LM head and verify + commit only."""
         ob = self.ob
         ev = events or {}
         if "t0" in ev:
             ev["t0"].record(stream)
-        for i in range(self.layers):
-            ob.block_attn(self.q_diff[i], None, None, None, ob.MASK_DIFF, out=self.attn_out,
-                          workspace=self.ws_attn, dev_status=self.status, stream=stream,
-                          cache_view=self.views[i])
+        if not verify_only:
+            for i in range(self.layers):
+                ob.block_attn(self.q_diff[i], None, None, None, ob.MASK_DIFF, out=self.attn_out,
+                              workspace=self.ws_attn, dev_status=self.status, stream=stream,
+                              cache_view=self.views[i])
         if "t1" in ev:
             ev["t1"].record(stream)
-        ob.lmhead_argmax(self.h_diff, self.W, argmax=self.draft, workspace=self.ws_lm,
-                         stream=stream, dev_status=self.status)
+        if not verify_only:
+            ob.lmhead_argmax(self.h_diff, self.W, argmax=self.draft, workspace=self.ws_lm,
+                             stream=stream, dev_status=self.status)
         if "t2" in ev:
             ev["t2"].record(stream)
         for i in range(self.layers):
@@ -310,7 +342,7 @@ class Workload:
             ev["t5"].record(stream)
 
 
-def capture(wl: Workload, n_steps: int, stream, with_events: bool):
+def capture(wl: Workload, n_steps: int, stream, with_events: bool, verify_only=False):
     """CUDA graph of n_steps unrolled steps (+ external timing events per phase)."""
     import torch
     evs = []
@@ -322,7 +354,7 @@ def capture(wl: Workload, n_steps: int, stream, with_events: bool):
                 e = {k: torch.cuda.Event(enable_timing=True, external=True)
                      for k in ("t0", "t1", "t2", "t3", "t4", "t5")}
                 evs.append(e)
-            wl.step(stream, e)
+            wl.step(stream, e, verify_only=verify_only)
     return g, evs
 
 
@@ -417,6 +449,11 @@ def run_ours(args):
         "steps": K_steps,
         "warmup": W_steps,
         "ms_per_step": round(ms_step, 4),
+        "value_counts": "verified draft positions: B*K per step, every block position scored "
+                        "by the AR pass and compared with its draft",
+        "emitted_tokens_per_s": round(weak_scaling_value(wl.emitted_per_step(), world, ms_step),
+                                      2),
+        "emitted_per_step": wl.emitted_per_step(),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -446,7 +483,8 @@ def run_ours(args):
         "lmhead": {"us_per_call": round(lm_us, 2), "GB_per_s": round(lm_gbs, 1),
                    "TFLOP_per_s": round(lm_tflops, 1),
                    "frac_of_hbm_peak": round(lm_gbs / hbm_peak, 4),
-                   "frac_of_bf16_peak": round(lm_tflops / tc_sus, 4)},
+                   "frac_of_bf16_peak": round(lm_tflops / tc_sus, 4),
+                   "frac_of_bf16_peak_burst": round(lm_tflops / tc_peak, 4)},
         "roofline": {
             "kernel": "orthrus_block_attn (cooperative split-KV kernel with in-kernel LSE merge), "
                       "AR and DIFF masks",
@@ -469,8 +507,15 @@ def run_ours(args):
         result["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl.L0, wl.K, wl.layers)
-    if args.sweep and rank == 0:
-        result["sweep"] = run_sweep(dev, stream)
+    if world == 1 and not args.no_extras:
+        del wl
+        torch.cuda.empty_cache()
+        result["ragged_batch"] = run_ragged(dev, stream, hbm_peak, tc_peak, tc_sus)
+        result["sweep"] = run_sweep(dev, stream, hbm_peak)
+        try:  # a separate kernel; its failure is reported, not fatal to the step's line
+            result["prefill"] = run_prefill(dev, stream, tc_peak)
+        except Exception as exc:  # noqa: BLE001
+            result["prefill"] = {"error": f"{type(exc).__name__}: {exc}"}
     if world > 1:
         sync_ranks()
         dist.destroy_process_group()
@@ -558,39 +603,154 @@ def run_e2e(wl: Workload, g_step, stream, K_steps, W_steps, world, dev):
     wall_ms = (time.perf_counter() - t0) * 1e3 / K_steps
     return {"value": round(weak_scaling_value(wl.B * wl.K, world, ms), 2), "unit": UNIT,
             "ms_per_step": round(ms, 4), "host_wall_ms_per_step": round(wall_ms, 4),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "how": "per step: one pinned host->device copy of every input of the step (both "
+                   "views' queries for all 72 layer calls and both views' final hidden states), "
+                   "a replay of the CUDA graph in which the step's C-ABI calls were recorded "
+                   "once, and a device->host read of accept lengths, next tokens and lengths; "
+                   "each step synchronised"}
 
 
-def run_sweep(dev, stream):
-    """Config 5 sweep: AR-pass step time for K x L (36 layers, batch 1)."""
+def time_graph_steps(wl: Workload, stream, n_steps: int, verify_only=False, replays=3):
+    """Per-phase device times (ms, averaged over steps) of n_steps unrolled steps
+    in one CUDA graph, after an eager step and a warm replay; the committed
+    lengths are reset before every replay."""
+    import torch
+    with torch.cuda.stream(stream):
+        wl.step(stream, verify_only=verify_only)
+        stream.synchronize()
+        g, evs = capture(wl, n_steps, stream, with_events=True, verify_only=verify_only)
+    ph = None
+    for _ in range(replays):
+        with torch.cuda.stream(stream):
+            wl.ctx_lens.copy_(wl.ctx_init)
+            g.replay()
+        torch.cuda.synchronize()
+        cur = {"diff_attn": 0.0, "diff_lm": 0.0, "ar_attn": 0.0, "ar_lm": 0.0, "verify": 0.0,
+               "step": 0.0}
+        for e in evs:
+            cur["diff_attn"] += e["t0"].elapsed_time(e["t1"])
+            cur["diff_lm"] += e["t1"].elapsed_time(e["t2"])
+            cur["ar_attn"] += e["t2"].elapsed_time(e["t3"])
+            cur["ar_lm"] += e["t3"].elapsed_time(e["t4"])
+            cur["verify"] += e["t4"].elapsed_time(e["t5"])
+            cur["step"] += e["t0"].elapsed_time(e["t5"])
+        cur = {k: v / len(evs) for k, v in cur.items()}
+        ph = cur  # the last replay is reported (the earlier ones are warm-up)
+    del g, evs
+    return ph
+
+
+def run_ragged(dev, stream, hbm_peak, tc_peak, tc_sus, n_steps=8):
+    """The ragged-batch configuration: 8 sequences with committed lengths uniform
+    in [1024, 32768], K = 32, per-sequence planted accept lengths uniform in
+    0..32, the full dual-view step over 36 layers (the LM head then has
+    R = 256 rows); the commit advances each sequence by min(accept + 1, 32)."""
+    import torch
+    from lossless_block_drafting_b200 import synth
+    B, K = 8, 32
+    lens = [int(x) for x in synth.ctx_lens_uniform(B, 1024, 32768, seed=4)]
+    accepts = [int(x) for x in synth.accept_uniform(B, K, seed=5)]
+    wl = Workload(B, K, lens, QWEN["layers"], accepts, n_steps + 4, dev, seed=77)
+    ph = time_graph_steps(wl, stream, n_steps)
+    got_accept = wl.accept_len.cpu().tolist()
+    attn_us = (ph["diff_attn"] + ph["ar_attn"]) * 1e3 / (2 * wl.layers)
+    lm_us = (ph["diff_lm"] + ph["ar_lm"]) * 1e3 / 2
+    attn_gbs = wl.attn_bytes() / (attn_us * 1e-6) / 1e9
+    lm_tf = wl.lm_flops() / (lm_us * 1e-6) / 1e12
+    out = {
+        "config": "8 sequences, committed lengths U[1024, 32768] (seed 4), K 32, 36 layers, "
+                  "32q/8kv d128, vocab 151936; planted accept lengths U{0..32} (seed 5)",
+        "ctx_lens": lens, "accept_planted": accepts, "accept_device": got_accept,
+        "ms_per_step": round(ph["step"], 4),
+        "verified_tokens_per_s": round(B * K / (ph["step"] * 1e-3), 1),
+        "emitted_tokens_per_s": round(wl.emitted_per_step() / (ph["step"] * 1e-3), 1),
+        "breakdown_ms_per_step": {k: round(v, 4) for k, v in ph.items() if k != "step"},
+        "attn": {"us_per_call": round(attn_us, 2), "GB_per_s": round(attn_gbs, 1),
+                 "frac_of_hbm_peak": round(attn_gbs / hbm_peak, 4)},
+        "lmhead_r256": {"us_per_call": round(lm_us, 2), "TFLOP_per_s": round(lm_tf, 1),
+                        "frac_of_bf16_peak_burst": round(lm_tf / tc_peak, 4),
+                        "frac_of_bf16_peak_sustained": round(lm_tf / tc_sus, 4),
+                        "GB_per_s": round(wl.lm_bytes() / (lm_us * 1e-6) / 1e9, 1)},
+        "device_status": int(wl.status.item()),
+    }
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_prefill(dev, stream, tc_peak, launches=4):
+    """The AR view's pre-filling pass: causal attention over a whole prompt of P
+    tokens (batch 1, 32 query / 8 KV heads, head_dim 128), one layer, timed
+    alone in a CUDA graph of back-to-back launches.  Flops = 4 * Hq * d * sum
+    over rows of the keys each row attends (i + 1 for row i): the masked-out
+    upper triangle is not counted."""
+    import torch
+    from lossless_block_drafting_b200 import orthrus as ob
+    out = []
+    Hq, Hkv, d = QWEN["Hq"], QWEN["Hkv"], QWEN["d"]
+    for P in (4096, 32768):
+        g = torch.Generator(device=dev).manual_seed(P)
+        q = torch.randn(1, P, Hq, d, generator=g, device=dev).to(torch.bfloat16)
+        kc = torch.randn(1, Hkv, P, d, generator=g, device=dev).to(torch.bfloat16)
+        vc = torch.randn(1, Hkv, P, d, generator=g, device=dev).to(torch.bfloat16)
+        cl = torch.zeros(1, dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        view = ob.kv_cache_view(kc, vc, cl)
+        with torch.cuda.stream(stream):
+            ob.prefill_attn(q, None, None, None, out=o, dev_status=st, stream=stream,
+                            cache_view=view)
+            stream.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for _ in range(launches):
+                    ob.prefill_attn(q, None, None, None, out=o, dev_status=st, stream=stream,
+                                    cache_view=view)
+            gr.replay()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            gr.replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+        us = t0.elapsed_time(t1) * 1e3 / launches
+        flops = 4.0 * Hq * d * P * (P + 1) / 2
+        tf = flops / (us * 1e-6) / 1e12
+        out.append({"P": P, "us_per_call": round(us, 1), "TFLOP_per_s": round(tf, 1),
+                    "frac_of_bf16_peak_burst": round(tf / tc_peak, 4),
+                    "device_status": int(st.item())})
+        del gr, q, kc, vc, o
+        torch.cuda.empty_cache()
+    return {"workload": "whole-prompt causal attention, batch 1, 32q/8kv d128, one layer",
+            "points": out, "bound": "tensor"}
+
+
+def run_sweep(dev, stream, hbm_peak, n_steps=4):
+    """The verify-step sweep: K in {1, 4, 8, 16, 32} x context in {1024, 8192,
+    40960, 131072}, batch 1, 36 layers: per point the AR pass (36 block
+    attentions), the LM head + argmax and verify + commit, from a CUDA graph of
+    n_steps steps.  One set of caches per context serves every K."""
     import torch
     out = []
     for L in (1024, 8192, 40960, 131072):
+        base = Workload(1, 32, L, QWEN["layers"], 0, n_steps + 4, dev, seed=7)
+        kv = (base.k, base.v)
         for K in (1, 4, 8, 16, 32):
-            layers = QWEN["layers"]
-            wl = Workload(1, K, L, layers, 0, 12, dev, seed=7)
-            with torch.cuda.stream(stream):
-                wl.step(stream)
-                stream.synchronize()
-                g, evs = capture(wl, 5, stream, with_events=True)
-            with torch.cuda.stream(stream):
-                for _ in range(2):
-                    wl.ctx_lens.copy_(wl.ctx_init)
-                    g.replay()
-            torch.cuda.synchronize()
-            ar = sum(e["t2"].elapsed_time(e["t3"]) for e in evs) / len(evs)
-            lm = sum(e["t3"].elapsed_time(e["t4"]) for e in evs) / len(evs)
-            vc = sum(e["t4"].elapsed_time(e["t5"]) for e in evs) / len(evs)
-            full = sum(e["t0"].elapsed_time(e["t5"]) for e in evs) / len(evs)
-            attn_us = ar * 1e3 / layers
-            out.append({"ctx": L, "K": K,
-                        "verify_step_ms": round(ar + lm + vc, 4),
-                        "full_step_ms": round(full, 4),
-                        "attn_us": round(attn_us, 2),
-                        "attn_GB_per_s": round(wl.attn_bytes() / (attn_us * 1e-6) / 1e9, 1),
-                        "verified_tok_per_s": round(K / ((ar + lm + vc) * 1e-3), 1)})
-            del g, evs, wl
-            torch.cuda.empty_cache()
+            wl = base if K == 32 else Workload(1, K, L, QWEN["layers"], 0, n_steps + 4, dev,
+                                               seed=7 + K, kv=kv)
+            ph = time_graph_steps(wl, stream, n_steps, verify_only=True)
+            verify_ms = ph["ar_attn"] + ph["ar_lm"] + ph["verify"]
+            attn_us = ph["ar_attn"] * 1e3 / wl.layers
+            gbs = wl.attn_bytes() / (attn_us * 1e-6) / 1e9
+            out.append({"ctx": L, "K": K, "verify_step_ms": round(verify_ms, 4),
+                        "attn_us": round(attn_us, 2), "attn_GB_per_s": round(gbs, 1),
+                        "attn_frac_of_hbm_peak": round(gbs / hbm_peak, 4),
+                        "lmhead_us": round(ph["ar_lm"] * 1e3, 2),
+                        "verified_tokens_per_s": round(K / (verify_ms * 1e-3), 1)})
+            if wl is not base:
+                del wl
+        del base, kv
+        torch.cuda.empty_cache()
     return out
 
 

@@ -162,6 +162,35 @@ int orthrus_block_attn(const void *q, const orthrus_kv_cache *cache, int Hq, int
                        int32_t *dev_status, void *stream);
 
 /*
+ * Causal attention over a prompt chunk: the AR view's pre-filling pass
+ * ([GIST 2.1] item 1: the frozen AR head's only job is to pre-fill the context
+ * into the shared cache both views read; [ABS]: the autoregressive head
+ * executes context pre-filling).
+ *
+ * For sequence b with L_b = ctx_lens[b], chunk row i in [0, P) at position
+ * L_b + i, query head h, KV head g = h / (Hq / Hkv):
+ *     out[b,i,h,:] = sum_j softmax(s)_j * v[b,g,j,:],
+ *     s_j = (q[b,i,h,:] . k[b,g,j,:]) / sqrt(d),   j < L_b + i + 1
+ * -- orthrus_block_attn's AR mask with the chunk in place of the block (L_b = 0
+ * for a whole prompt, L_b > 0 for a later chunk of a long one), bf16 inputs,
+ * fp32 accumulation and softmax, bf16 output.
+ *   q          bf16 [B, P, Hq, d] device (post-RoPE queries of the chunk)
+ *   cache      KV cache view; the caller has written the chunk's K/V into slots
+ *              [L_b, L_b + P) (orthrus_block_qkv_append with K = P does so with
+ *              the Qwen3 epilogue).  ctx_lens is read, not changed: advance it
+ *              by P afterwards.
+ *   Hq, P      query heads (multiple of cache->Hkv), chunk length (>= 1)
+ *   out        bf16 [B, P, Hq, d] device
+ *   dev_status int32 device or NULL: ORTHRUS_ECAPACITY when L_b + P > cap
+ *              (L_b is then clamped to cap - P)
+ * Supported: d in {64, 128}.  No workspace.  One CTA per pair of query heads of
+ * a KV group and 128 positions (tcgen05 MMAs, TMEM accumulators, TMA-staged
+ * Q/K/V), latest positions first.
+ */
+int orthrus_prefill_attn(const void *q, const orthrus_kv_cache *cache, int Hq, int P, void *out,
+                         int32_t *dev_status, void *stream);
+
+/*
  * Workspace bytes orthrus_lmhead_argmax needs on the CURRENT device.
  */
 int orthrus_lmhead_workspace_size(int R, int V, size_t *bytes);

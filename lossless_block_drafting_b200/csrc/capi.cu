@@ -118,7 +118,7 @@ extern "C" const char* orthrus_status_str(int status) {
   }
 }
 
-extern "C" int orthrus_abi_version(void) { return 2; }
+extern "C" int orthrus_abi_version(void) { return 3; }
 
 extern "C" int orthrus_set_wait_limit_ns(uint64_t ns) {
   orthrus::g_wait_ns.store(ns == 0 ? orthrus::kDefaultWaitNs : ns, std::memory_order_relaxed);

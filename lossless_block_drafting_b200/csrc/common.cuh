@@ -76,6 +76,18 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
+// Wait that ignores the abort flag, used only to let in-flight asynchronous
+// work (copies, MMAs) finish before the CTA exits; gives up after 200 ms.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, int32_t* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) {
+      report(status, ORTHRUS_ETIMEOUT);
+      return;
+    }
+  }
+}
+
 // max(a, b, c) in one instruction (three-input form of max.f32).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

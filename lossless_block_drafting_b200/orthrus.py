@@ -60,6 +60,7 @@ def load(path: str | None = None):
             "orthrus_set_wait_limit_ns": ([ctypes.c_uint64], I),
             "orthrus_block_attn_workspace_size": ([I, I, I, I, I, PSZ], I),
             "orthrus_block_attn": ([V, PC, I, I, I, V, V, SZ, V, V], I),
+            "orthrus_prefill_attn": ([V, PC, I, I, V, V, V], I),
             "orthrus_lmhead_workspace_size": ([I, I, PSZ], I),
             "orthrus_lmhead_argmax": ([V, V, I, I, I, V, V, V, SZ, V, V], I),
             "orthrus_lmhead_argmax_noalloc": ([V, V, I, I, I, V, V, V, V], I),
@@ -158,6 +159,27 @@ def block_attn(q, k_cache, v_cache, ctx_lens, mask_mode: int, out=None, workspac
                                    _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                    _stream(stream))
     _check(rc, "orthrus_block_attn")
+    return out
+
+
+def prefill_attn(q, k_cache, v_cache, ctx_lens, out=None, dev_status=None, stream=None,
+                 cache_view: KVCacheView | None = None):
+    """Causal attention of a prompt chunk q bf16 [B, P, Hq, d] at positions
+    ctx_lens[b] + i over the cache -> bf16 [B, P, Hq, d] (ctx_lens unchanged)."""
+    _need(q, torch.bfloat16, "q", 4)
+    view = cache_view if cache_view is not None else kv_cache_view(k_cache, v_cache, ctx_lens)
+    B, P, Hq, d = q.shape
+    if B != view.B or d != view.d:
+        raise ValueError("q must be [B, P, Hq, d] of the cache's B and d")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, torch.bfloat16, "out", 4)
+    if dev_status is not None:
+        _need(dev_status, torch.int32, "dev_status")
+    rc = load().orthrus_prefill_attn(_ptr(q), ctypes.byref(view), Hq, P, _ptr(out),
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "orthrus_prefill_attn")
     return out
 
 

@@ -31,7 +31,7 @@ def test_header_declares_the_boundary():
                  "orthrus_kv_commit", "orthrus_verify_commit", "orthrus_row_argmax_f32",
                  "orthrus_block_attn_workspace_size", "orthrus_lmhead_workspace_size",
                  "orthrus_status_str", "orthrus_abi_version", "orthrus_block_qkv_append",
-                 "orthrus_set_wait_limit_ns"):
+                 "orthrus_set_wait_limit_ns", "orthrus_prefill_attn"):
         assert want in names
 
 
@@ -45,7 +45,7 @@ def test_status_strings(lib):
         s = ob.status_str(code)
         assert s.startswith("ORTHRUS")
     assert "unknown" in ob.status_str(-99)
-    assert lib.orthrus_abi_version() == 2
+    assert lib.orthrus_abi_version() == 3
 
 
 def test_wait_limit_setter_accepts_any_value(lib):
@@ -142,3 +142,23 @@ def test_qkv_append_host_validation(lib):
     assert f(*args(K=65)) == ob.ESHAPE                     # cap < K
     assert f(*args(out=A + 2)) == ob.EALIGN
     assert f(*args(view=_view(B=0, Hkv=2, cap=64, d=128))) == ob.OK
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(P=0), ob.EINVAL),
+    (dict(Hq=3), ob.ESHAPE),            # Hq % Hkv != 0
+    (dict(d=96), ob.EUNSUPPORTED),
+    (dict(cap=16, P=32), ob.ESHAPE),    # cap < P
+    (dict(q=A + 8), ob.EALIGN),
+    (dict(q=None), ob.EINVAL),
+])
+def test_prefill_attn_host_validation(lib, kwargs, status):
+    view = _view(cap=kwargs.get("cap", 64), d=kwargs.get("d", 64))
+    rc = lib.orthrus_prefill_attn(kwargs.get("q", A), ctypes.byref(view), kwargs.get("Hq", 4),
+                                  kwargs.get("P", 8), A, None, None)
+    assert rc == status
+
+
+def test_prefill_attn_empty_batch_is_a_noop(lib):
+    view = _view(B=0)
+    assert lib.orthrus_prefill_attn(A, ctypes.byref(view), 4, 8, A, None, None) == ob.OK
