@@ -18,12 +18,11 @@
 // columns), the longest (latest) position tiles launched first.
 //   warp 0      TMA: both Q tiles once, then K and V groups into 2-stage rings.
 //   warp 1      the single tcgen05 issuer, in the order
-//                 S0(0) S1(0) | PV0(j) PV1(j) S0(j+1) S1(j+1) | ...
-//               so the tensor core computes one tile while the other tile's
-//               softmax runs.  S_t and P_t share tile t's 128 TMEM columns
-//               (P overwrites the first 64 as bf16), so S_t(j+1) is issued
-//               only once PV_t(j) has completed (PV_(1-t) keeps the tensor
-//               core busy meanwhile).
+//                 S0(0) S1(0) | PV0(j) S0(j+1) PV1(j) S1(j+1) | ...
+//               S_t and P_t share tile t's 128 TMEM columns (P overwrites the
+//               first 64 as bf16), so S_t(j+1) is issued once PV_t(j) has
+//               completed.  The two tiles settle half a period apart: the
+//               tensor core works on one while the other's softmax runs.
 //   warp 2      TMEM allocation.
 //   warps 4-7   softmax of tile 0, warps 8-11 of tile 1: one thread per row,
 //               64 keys at a time, exp2 against a running reference maximum
@@ -239,24 +238,25 @@ __global__ void __launch_bounds__(THREADS, 1)
       mma_commit(k_empty(0));
       for (int j = 0; ok && j < ngroups; ++j) {
         const int s = j % NST;
+        const bool more = j + 1 < ngroups;
         WAIT_OR(v_full(s), (j / NST) & 1, { ok = false; break; });
         for (int t = 0; t < nt; ++t) {
+          // tile t: P_t(j) -> PV_t(j); once it has consumed P_t(j), S_t(j + 1)
+          // may overwrite it.  The other tile's softmax runs meanwhile, so
+          // the two tiles settle half a period apart.
           WAIT_OR(p_full(t), j & 1, { ok = false; break; });
           tc_fence_after();
           issue_pv(t, j);
-        }
-        if (!ok) break;
-        mma_commit(v_empty(s));
-        if (j + 1 < ngroups) {
-          WAIT_OR(k_full((j + 1) % NST), ((j + 1) / NST) & 1, { ok = false; break; });
-          for (int t = 0; t < nt; ++t) {
-            // S_t(j + 1) overwrites P_t(j): only after PV_t(j) has completed
+          if (t == nt - 1) mma_commit(v_empty(s));
+          if (more) {
+            if (t == 0) {
+              WAIT_OR(k_full((j + 1) % NST), ((j + 1) / NST) & 1, { ok = false; break; });
+            }
             WAIT_OR(pv_done(t), j & 1, { ok = false; break; });
             tc_fence_after();
             issue_s(t, j + 1);
+            if (t == nt - 1) mma_commit(k_empty((j + 1) % NST));
           }
-          if (!ok) break;
-          mma_commit(k_empty((j + 1) % NST));
         }
       }
     } while (0);
