@@ -220,7 +220,8 @@ class Workload:
     optional (k, v) lists of per-layer caches to share with another workload.
     """
 
-    def __init__(self, B, K, lens, layers, accepts, steps_total, device, seed=0, kv=None):
+    def __init__(self, B, K, lens, layers, accepts, steps_total, device, seed=0, kv=None,
+                 with_append=False):
         import torch
         from lossless_block_drafting_b200 import orthrus as ob
         self.ob = ob
@@ -281,12 +282,21 @@ class Workload:
         self.next_tok = torch.empty(B, dtype=torch.int32, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.views = [ob.kv_cache_view(self.k[i], self.v[i], self.ctx_lens) for i in range(layers)]
+        # With the block Q/K/V append in the step, every layer call first turns
+        # that view's packed projections into rotated queries (written over
+        # q_diff / q_ar) and the block's K/V in cache slots [L_b, L_b + K).
+        self.with_append = with_append
+        if with_append:
+            W = Hq + 2 * Hkv
+            self.qkv_diff = [randn(B * K, W * d) for _ in range(layers)]
+            self.qkv_ar = [randn(B * K, W * d) for _ in range(layers)]
+            self.qk_w = (1.0 + 0.1 * torch.randn(2, d, generator=g, device=device)).to(bf)
 
     # kernels launched per step (one per attention call; main + reduce per LM
     # head; one verify+commit)
     @property
     def launches_per_step(self):
-        return 2 * self.layers + 2 * 2 + 1
+        return (4 if self.with_append else 2) * self.layers + 2 * 2 + 1
 
     def emitted_per_step(self):
         """Tokens a step emits: the accepted drafts plus the correction (or the
@@ -306,6 +316,11 @@ class Workload:
     def lm_flops(self):
         return 2.0 * self.B * self.K * self.H * self.V
 
+    def append(self, qkv, q_out, i, stream):
+        self.ob.block_qkv_append(qkv, None, None, None, self.Hq, self.K, q_norm_w=self.qk_w[0],
+                                 k_norm_w=self.qk_w[1], q_out=q_out, cache_view=self.views[i],
+                                 dev_status=self.status, stream=stream)
+
     def step(self, stream, events=None, verify_only=False):
         """Issue one decode step on `stream`; events (if given) mark phase
         boundaries.  verify_only: the AR pass, LM head and verify + commit only."""
@@ -315,6 +330,8 @@ class Workload:
             ev["t0"].record(stream)
         if not verify_only:
             for i in range(self.layers):
+                if self.with_append:
+                    self.append(self.qkv_diff[i], self.q_diff[i], i, stream)
                 ob.block_attn(self.q_diff[i], None, None, None, ob.MASK_DIFF, out=self.attn_out,
                               workspace=self.ws_attn, dev_status=self.status, stream=stream,
                               cache_view=self.views[i])
@@ -326,6 +343,8 @@ class Workload:
         if "t2" in ev:
             ev["t2"].record(stream)
         for i in range(self.layers):
+            if self.with_append:
+                self.append(self.qkv_ar[i], self.q_ar[i], i, stream)
             ob.block_attn(self.q_ar[i], None, None, None, ob.MASK_AR, out=self.attn_out,
                           workspace=self.ws_attn, dev_status=self.status, stream=stream,
                           cache_view=self.views[i])
@@ -510,6 +529,8 @@ def run_ours(args):
     if world == 1 and not args.no_extras:
         del wl
         torch.cuda.empty_cache()
+        result["step_with_append"] = run_step_with_append(dev, stream, args.ctx, args.block,
+                                                          args.layers, args.accept)
         result["ragged_batch"] = run_ragged(dev, stream, hbm_peak, tc_peak, tc_sus)
         result["sweep"] = run_sweep(dev, stream, hbm_peak)
         try:  # a separate kernel; its failure is reported, not fatal to the step's line
@@ -674,6 +695,29 @@ def run_ragged(dev, stream, hbm_peak, tc_peak, tc_sus, n_steps=8):
                         "GB_per_s": round(wl.lm_bytes() / (lm_us * 1e-6) / 1e9, 1)},
         "device_status": int(wl.status.item()),
     }
+    del wl
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_step_with_append(dev, stream, L, K, layers, accept, n_steps=8):
+    """The headline step with the block Q/K/V append (per-head RMS norm of q and
+    k, rotary embedding at L_b + i, block K/V into the cache) before each of its
+    72 attention calls, against the same workload's step without it (both from
+    the same graph timing): the append's cost inside the step."""
+    import torch
+    wl = Workload(1, K, L, layers, accept, n_steps + 4, dev, seed=1234, with_append=True)
+    with_app = time_graph_steps(wl, stream, n_steps)
+    wl.with_append = False
+    without = time_graph_steps(wl, stream, n_steps)
+    wl.with_append = True
+    out = {"ms_per_step": round(with_app["step"], 4),
+           "ms_per_step_without_append": round(without["step"], 4),
+           "verified_tokens_per_s": round(K / (with_app["step"] * 1e-3), 1),
+           "append_us_per_call_in_step": round(
+               (with_app["step"] - without["step"]) * 1e3 / (2 * layers), 2),
+           "launches_per_step": wl.launches_per_step,
+           "device_status": int(wl.status.item())}
     del wl
     torch.cuda.empty_cache()
     return out

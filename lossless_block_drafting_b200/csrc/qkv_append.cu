@@ -7,12 +7,14 @@
 // per-head RMS normalisation of q and k, then the rotary position embedding
 // with coordinate j paired with j + d/2 and angle (L_b + i) * theta^(-2j/d).
 //
-// One CTA per block token: the d/2 angles are evaluated in double precision
-// (exact for any position up to 2^31) and kept as fp32 (cos, sin) pairs in
-// shared memory; each warp then takes whole heads, lane l holding elements
-// l, l + 32, ... so both members of every rotated pair sit in the same lane.
-// The step moves (Hq + 2 Hkv) d bf16 in and out per token: latency-bound at
-// decode sizes.
+// One CTA per (block token, group of 8 heads), one warp per head (a
+// Qwen3-8B block of 32 tokens and 48 heads is 192 CTAs): the d/2 angles
+// p * theta^(-2j/d) are evaluated in double precision from inverse
+// frequencies the host computes once (exact for any position up to 2^31) and
+// kept as fp32 (cos, sin) pairs in shared memory; lane l of a warp holds
+// elements l, l + 32, ... of its head, so both members of every rotated pair
+// sit in the same lane.  The step moves (Hq + 2 Hkv) d bf16 in and out per
+// token: latency-bound at decode sizes.
 #include <cmath>
 
 #include "common.cuh"
@@ -21,7 +23,9 @@
 namespace orthrus {
 namespace qkv {
 
-constexpr int THREADS = 256;
+constexpr int HPB = 8;                  // heads (warps) per CTA
+constexpr int THREADS = HPB * 32;
+constexpr int MAX_HALF = 64;            // d / 2 for d <= 128
 
 struct Params {
   const __nv_bfloat16* qkv;   // [B*K, (Hq + 2 Hkv) d]
@@ -32,9 +36,9 @@ struct Params {
   __nv_bfloat16* vc;
   const int32_t* ctx_lens;
   int32_t* dev_status;
-  int K, Hq, Hkv, cap;
-  double theta;
+  int K, Hq, Hkv, cap, ngrp;
   float eps;
+  double inv_freq[MAX_HALF];  // theta^(-2j/d), j < d/2
 };
 
 template <int D>
@@ -43,7 +47,7 @@ __global__ void __launch_bounds__(THREADS) qkv_append_kernel(const Params p) {
   __shared__ float2 cs[D / 2];
   grid_dep_launch();
   grid_dep_wait();  // qkv, ctx_lens and the cache may come from the previous kernel
-  const int t = blockIdx.x;
+  const int t = blockIdx.x / p.ngrp, grp = blockIdx.x % p.ngrp;
   const int b = t / p.K, i = t - b * p.K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int L = __ldg(p.ctx_lens + b);
@@ -54,14 +58,15 @@ __global__ void __launch_bounds__(THREADS) qkv_append_kernel(const Params p) {
   }
   const int pos = L + i;
   for (int j = threadIdx.x; j < D / 2; j += THREADS) {
-    const double a = static_cast<double>(pos) * pow(p.theta, -2.0 * j / D);
+    const double a = static_cast<double>(pos) * p.inv_freq[j];
     double s, c;
     sincos(a, &s, &c);
     cs[j] = make_float2(static_cast<float>(c), static_cast<float>(s));
   }
   __syncthreads();
   const int W = p.Hq + 2 * p.Hkv;
-  for (int hh = warp; hh < W; hh += THREADS / 32) {
+  const int hh = grp * HPB + warp;
+  if (hh < W) {
     const __nv_bfloat16* src = p.qkv + (static_cast<long long>(t) * W + hh) * D;
     float x[E];
 #pragma unroll
@@ -137,9 +142,13 @@ extern "C" int orthrus_block_qkv_append(const void* qkv, const void* q_norm_w,
   p.Hq = Hq;
   p.Hkv = cache->Hkv;
   p.cap = cache->cap;
-  p.theta = static_cast<double>(rope_theta);
   p.eps = rms_eps;
-  const dim3 grid(static_cast<unsigned>(cache->B * K));
+  p.ngrp = (Hq + 2 * cache->Hkv + qkv::HPB - 1) / qkv::HPB;
+  for (int j = 0; j < cache->d / 2; ++j)
+    p.inv_freq[j] = std::pow(static_cast<double>(rope_theta), -2.0 * j / cache->d);
+  const long long nblk = static_cast<long long>(cache->B) * K * p.ngrp;
+  if (nblk >= (1ll << 31)) return ORTHRUS_EUNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(nblk));
   const cudaStream_t s = as_stream(stream);
   if (cache->d == 128)
     return launch_kernel(qkv::qkv_append_kernel<128>, grid, dim3(qkv::THREADS), 0, s, p);
