@@ -428,27 +428,26 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, i
 // never needs resetting); the generation is complete once the counter reaches
 // the next multiple.  Bounded: a wait that gives up reports ETIMEOUT.
 // grid_wait compares by signed difference, so a counter that wraps past 2^64
-// still reaches its target.
+// still reaches its target.  Release on arrival (the CTA barrier before it
+// orders the other threads' writes), acquire by the polling load.
 __device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* gbar,
                                                           unsigned int nctas) {
-  __threadfence();
+  fence_acq_rel_gpu();
   const unsigned long long ticket = atomicAdd(gbar, 1ull);
   return (ticket / nctas + 1) * nctas;
 }
 
 __device__ bool grid_wait(unsigned long long* gbar, unsigned long long target,
                           int32_t* status, uint64_t limit_ns) {
-  volatile unsigned long long* v = gbar;
   const uint64_t t0 = globaltimer_ns();
   bool ok = true;
-  for (uint32_t polls = 0; static_cast<long long>(*v - target) < 0; ++polls) {
+  for (uint32_t polls = 0; static_cast<long long>(ld_acquire_gpu(gbar) - target) < 0; ++polls) {
     if ((polls & 255u) == 255u && globaltimer_ns() - t0 > limit_ns) {
       report(status, ORTHRUS_ETIMEOUT);
       ok = false;
       break;
     }
   }
-  __threadfence();
   return ok;
 }
 
@@ -1437,7 +1436,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row1e = BR * static_cast<int>(mul_div(k + 1, nblk, own.cn));
     const int row1 = row1e < RV ? row1e : RV;
     if (threadIdx.x == 0) {
-      __threadfence();
+      fence_acq_rel_gpu();  // release this CTA's partial (written before the CTA barrier)
       const unsigned long long add = k == 0 ? (1ull << 20) - (own.cn - 1) : 1ull;
       const unsigned long long old = atomicAdd(p.seg_cnt + own.s, add);
       if (row1 > row0 &&

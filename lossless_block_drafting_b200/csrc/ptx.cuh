@@ -157,6 +157,21 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// ------------------------------------------------ release / acquire (gpu)
+// Release: every write that happens-before this fence in this CTA (other
+// threads' writes ordered before it by a CTA barrier included) becomes
+// visible at gpu scope before this thread's later writes.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+// Acquire load at gpu scope: later reads of this thread observe every write
+// released before the value it returns was written.
+__device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // ------------------------------------------ programmatic dependent launch
 // Lets the next kernel in the stream (launched with programmatic stream
 // serialisation) be scheduled once every CTA of this grid has issued it or
