@@ -10,7 +10,9 @@
 // Design (B200, sm_100a).  One KV head serves G = Hq/Hkv query heads, so the
 // G*K queries of a (sequence b, KV head g, head chunk hc) segment are packed
 // into one 128-row tcgen05 M tile (row r = i*Gc + hh) and every K/V byte is
-// read from HBM once.  One cooperative, persistent launch of one CTA per SM;
+// read from HBM once.  One persistent launch of one CTA per SM (cooperative,
+// or plain under programmatic dependent launch, which keeps every CTA
+// resident too: see the launch);
 // the keys of each segment are cut into 64-key tiles, loaded in groups of two
 // (one 128-row TMA box per 128-byte column chunk).
 //
@@ -66,6 +68,9 @@ constexpr int TN = 64;        // keys per compute tile
 // the TMA engines near HBM bandwidth (measured: 64-row boxes top out at about
 // 80% of it, 128-row boxes near 97%).
 constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
+// Load groups of its static run a CTA asks L2 to prefetch while it still waits
+// for the previous kernel in the stream (4 groups = 256 KB of K and V at D = 128).
+constexpr int PREFETCH_GROUPS = 4;
 // Partial O layout: [ROWS / BR row blocks][slot][D / 4 column quads][BR rows][4]
 // floats.  A warp's store of one column quad for its 32 rows covers four whole
 // 128-byte lines, and since the pieces of a segment occupy consecutive slots,
@@ -992,6 +997,38 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_proxy_async_smem();
   }
 
+  // L2 warm-up while the previous kernel drains.  Warp 0 guesses the CTA's
+  // first static load groups from the lengths as they read now (through L2
+  // only, so no line of them stays in L1 past the wait) and prefetches their
+  // K and V into L2.  A prefetch moves nothing into shared memory and writes
+  // nothing, so a stale length (one that kernel is still changing) or a wrong
+  // guess costs bandwidth, never a result; the schedule itself is computed
+  // again after the wait.  Rows past the cache view are dropped by the tensor
+  // map's bounds.
+  if (warp == 0 && p.B <= 32 && p.balance) {
+    warp_schedule_small(p, gridDim.x, blockIdx.x, lane, false, sched,
+                        lane < p.B ? __ldcg(p.ctx_lens + lane) : 0);
+    __syncwarp();
+    if (lane == 0) {
+      const OwnSeg g0 = read_own();
+      if (g0.s >= 0 && g0.cn > 0) {
+        const int k = static_cast<int>(blockIdx.x) - g0.c0;
+        const int fs = static_cast<int>(mul_div(3 * ((g0.ns + 1) / 2), 1, 4 * g0.cn));
+        const int b = static_cast<int>(g0.s) / nseg, seg = static_cast<int>(g0.s) - b * nseg;
+        const int kvbase = (b * p.Hkv + seg / p.nhc) * p.cap;
+        const int n = fs < PREFETCH_GROUPS ? fs : PREFETCH_GROUPS;
+        for (int i = 0; i < n; ++i) {
+          const int row = kvbase + 2 * (k * fs + i) * TN;
+          for (int c = 0; c < Ly::CHUNKS; ++c) {
+            tma_prefetch_2d(&tmK2, c * 64, row);
+            tma_prefetch_2d(&tmV2, c * 64, row);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+
   grid_dep_wait();
   if (warp == 0) {
     warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
@@ -1568,30 +1605,60 @@ int launch(const Shape& sh, const void* q, const orthrus_kv_cache* cache, int ma
   auto* kfn = p.wait_ns < kShortWaitNs ? attn_splitkv_kernel<D, true>
                                        : attn_splitkv_kernel<D, false>;
   if (!opt_in_smem(reinterpret_cast<const void*>(kfn), Layout<D>::ALLOC)) return ORTHRUS_ECUDA;
-  // Cooperative launch: the grid barrier before the merge needs every CTA
-  // resident at once (one CTA per SM).  Programmatic stream serialisation lets
-  // the kernel's prologue overlap the tail of the previous kernel in the
-  // stream; the kernel waits (griddepcontrol.wait) before it reads anything
-  // that kernel may have written.
+  // The sibling wait and the grid barrier before the merge need every CTA of
+  // the grid resident at once (one CTA per SM; the shared memory allows no
+  // second).  Under programmatic dependent launch the launch is plain: this
+  // grid's CTAs then take SMs as the previous grid's CTAs exit, run their
+  // prologue (and the L2 warm-up) there and wait (griddepcontrol.wait) before
+  // they read anything that kernel may have written; a cooperative grid could
+  // only start once the previous grid had left every SM.  Residency still
+  // holds: every CTA triggers its dependents (griddepcontrol.launch_dependents)
+  // on entry, so a later grid of the stream is scheduled only once all of this
+  // grid's CTAs hold an SM, an earlier grid never waits on this one, and one
+  // CTA per SM fits (checked once below).  Kernels of other streams can still
+  // hold SMs while some CTAs wait for theirs; past the wait limit that ends the
+  // call with ETIMEOUT.  Callers that overlap other streams' kernels with
+  // attention set ORTHRUS_ATTN_COOPERATIVE (or ORTHRUS_NO_PDL): the launch is
+  // then cooperative, which the runtime starts only when the whole grid fits.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = Layout<D>::ALLOC;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  // If the runtime refuses the pair of attributes, the first (eager) call
-  // finds out and every later call launches cooperatively only.
+  cudaError_t e = cudaErrorNotSupported;
+  if (pdl_enabled() && !attn_cooperative()) {
+    static std::atomic<int> fits{-1};  // one CTA per SM fits: checked once
+    if (fits.load(std::memory_order_relaxed) < 0) {
+      int per_sm = 0;
+      const bool ok = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                          &per_sm, kfn, THREADS, Layout<D>::ALLOC) == cudaSuccess;
+      fits.store(ok && per_sm >= 1 ? 1 : 0, std::memory_order_relaxed);
+    }
+    if (fits.load(std::memory_order_relaxed) == 0) return ORTHRUS_ECUDA;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
+    if (e != cudaSuccess) return ORTHRUS_ECUDA;
+    return ORTHRUS_OK;
+  }
+  // Cooperative, with the programmatic attribute as well when it is on (the
+  // prologue then overlaps only the previous kernel's final flush).  If the
+  // runtime refuses the pair, the first (eager) call finds out and every later
+  // call launches cooperatively only.
   static std::atomic<bool> coop_pdl_ok{true};
-  cfg.numAttrs = (pdl_enabled() && coop_pdl_ok.load(std::memory_order_relaxed)) ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
-  if (e != cudaSuccess && cfg.numAttrs == 2) {
+  const bool pair = pdl_enabled() && coop_pdl_ok.load(std::memory_order_relaxed);
+  cfg.attrs = pair ? attr : attr + 1;
+  cfg.numAttrs = pair ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
+  if (e != cudaSuccess && pair) {
     (void)cudaGetLastError();
     coop_pdl_ok.store(false, std::memory_order_relaxed);
+    cfg.attrs = attr + 1;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kfn, tq, tk2, tk1, tv2, tv1, p);
   }

@@ -93,6 +93,11 @@ bool pdl_enabled() {
   return on;
 }
 
+bool attn_cooperative() {
+  static const bool on = std::getenv("ORTHRUS_ATTN_COOPERATIVE") != nullptr;
+  return on;
+}
+
 int current_sm_count(int* sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ORTHRUS_ECUDA;

@@ -39,6 +39,12 @@ uint64_t wait_limit_ns();
 // first launches a kernel).
 bool pdl_enabled();
 
+// Whether block attention always launches cooperatively (the environment
+// variable ORTHRUS_ATTN_COOPERATIVE is set when the library first launches
+// it): for callers that run other kernels concurrently on other streams, so
+// the grid starts only once every CTA can be resident.
+bool attn_cooperative();
+
 // Launch `kernel` on `s`, with the programmatic-stream-serialisation
 // attribute when pdl_enabled(); every kernel of this library calls
 // griddepcontrol.wait before it touches memory a preceding kernel may write.

@@ -8,6 +8,7 @@ path, and a missing library raises instead of falling back.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -98,6 +99,13 @@ def _stream(stream) -> int | None:
     return s.cuda_stream
 
 
+def _on(stream):
+    """Context for buffers a call allocates itself: on the launch stream, so a
+    zero fill is ordered before the kernel and the caching allocator reuses a
+    temporary only after that stream is done with it."""
+    return contextlib.nullcontext() if stream is None else torch.cuda.stream(stream)
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -147,12 +155,12 @@ def block_attn(q, k_cache, v_cache, ctx_lens, mask_mode: int, out=None, workspac
     _need(q, torch.bfloat16, "q", 4)
     view = cache_view if cache_view is not None else kv_cache_view(k_cache, v_cache, ctx_lens)
     B, K, Hq, d = q.shape
-    if out is None:
-        out = torch.empty_like(q)
-    else:
-        _need(out, torch.bfloat16, "out", 4)
-    if workspace is None:
-        workspace = new_block_attn_workspace(B, Hq, view.Hkv, d, K, q.device)
+    with _on(stream):
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            workspace = new_block_attn_workspace(B, Hq, view.Hkv, d, K, q.device)
+    _need(out, torch.bfloat16, "out", 4)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_block_attn(_ptr(q), ctypes.byref(view), Hq, K, int(mask_mode), _ptr(out),
@@ -172,9 +180,9 @@ def prefill_attn(q, k_cache, v_cache, ctx_lens, out=None, dev_status=None, strea
     if B != view.B or d != view.d:
         raise ValueError("q must be [B, P, Hq, d] of the cache's B and d")
     if out is None:
-        out = torch.empty_like(q)
-    else:
-        _need(out, torch.bfloat16, "out", 4)
+        with _on(stream):
+            out = torch.empty_like(q)
+    _need(out, torch.bfloat16, "out", 4)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_prefill_attn(_ptr(q), ctypes.byref(view), Hq, P, _ptr(out),
@@ -199,15 +207,17 @@ def lmhead_argmax(h, W, argmax=None, max_logit=None, workspace=None, stream=None
     V, H2 = W.shape
     if H2 != H:
         raise ValueError("h and W hidden sizes differ")
-    if argmax is None:
-        argmax = torch.empty(R, dtype=torch.int32, device=h.device)
+    with _on(stream):
+        if argmax is None:
+            argmax = torch.empty(R, dtype=torch.int32, device=h.device)
+        if want_max and max_logit is None:
+            max_logit = torch.empty(R, dtype=torch.float32, device=h.device)
+        if workspace is None:
+            workspace = torch.empty(lmhead_workspace_size(R, V), dtype=torch.uint8,
+                                    device=h.device)
     _need(argmax, torch.int32, "argmax", 1)
-    if want_max and max_logit is None:
-        max_logit = torch.empty(R, dtype=torch.float32, device=h.device)
     if max_logit is not None:
         _need(max_logit, torch.float32, "max_logit", 1)
-    if workspace is None:
-        workspace = torch.empty(lmhead_workspace_size(R, V), dtype=torch.uint8, device=h.device)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_lmhead_argmax(_ptr(h), _ptr(W), R, H, V, _ptr(argmax), _ptr(max_logit),
@@ -228,11 +238,12 @@ def lmhead_argmax_noalloc(h, W, argmax=None, max_logit=None, stream=None,
     V, H2 = W.shape
     if H2 != H:
         raise ValueError("h and W hidden sizes differ")
-    if argmax is None:
-        argmax = torch.empty(R, dtype=torch.int32, device=h.device)
+    with _on(stream):
+        if argmax is None:
+            argmax = torch.empty(R, dtype=torch.int32, device=h.device)
+        if want_max and max_logit is None:
+            max_logit = torch.empty(R, dtype=torch.float32, device=h.device)
     _need(argmax, torch.int32, "argmax", 1)
-    if want_max and max_logit is None:
-        max_logit = torch.empty(R, dtype=torch.float32, device=h.device)
     if max_logit is not None:
         _need(max_logit, torch.float32, "max_logit", 1)
     if dev_status is not None:
@@ -249,7 +260,8 @@ def row_argmax_f32(logits, argmax=None, stream=None):
     _need(logits, torch.float32, "logits", 2)
     R, V = logits.shape
     if argmax is None:
-        argmax = torch.empty(R, dtype=torch.int32, device=logits.device)
+        with _on(stream):
+            argmax = torch.empty(R, dtype=torch.int32, device=logits.device)
     _need(argmax, torch.int32, "argmax", 1)
     _check(load().orthrus_row_argmax_f32(_ptr(logits), R, V, _ptr(argmax), _stream(stream)),
            "orthrus_row_argmax_f32")
@@ -263,10 +275,11 @@ def verify(argmax, draft, accept_len=None, next_tok=None, stream=None):
     if argmax.shape != draft.shape:
         raise ValueError("argmax and draft shapes differ")
     B, K = argmax.shape
-    if accept_len is None:
-        accept_len = torch.empty(B, dtype=torch.int32, device=argmax.device)
-    if next_tok is None:
-        next_tok = torch.empty(B, dtype=torch.int32, device=argmax.device)
+    with _on(stream):
+        if accept_len is None:
+            accept_len = torch.empty(B, dtype=torch.int32, device=argmax.device)
+        if next_tok is None:
+            next_tok = torch.empty(B, dtype=torch.int32, device=argmax.device)
     _check(load().orthrus_verify(_ptr(argmax), _ptr(draft), B, K, _ptr(accept_len),
                                  _ptr(next_tok), _stream(stream)), "orthrus_verify")
     return accept_len, next_tok
@@ -294,10 +307,11 @@ def verify_commit(argmax, draft, ctx_lens, cap: int, accept_len=None, next_tok=N
     _need(argmax, torch.int32, "argmax", 2)
     _need(draft, torch.int32, "draft", 2)
     B, K = argmax.shape
-    if accept_len is None:
-        accept_len = torch.empty(B, dtype=torch.int32, device=argmax.device)
-    if next_tok is None:
-        next_tok = torch.empty(B, dtype=torch.int32, device=argmax.device)
+    with _on(stream):
+        if accept_len is None:
+            accept_len = torch.empty(B, dtype=torch.int32, device=argmax.device)
+        if next_tok is None:
+            next_tok = torch.empty(B, dtype=torch.int32, device=argmax.device)
     view = _lens_view(ctx_lens, cap)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
@@ -322,9 +336,9 @@ def block_qkv_append(qkv, k_cache, v_cache, ctx_lens, Hq: int, K: int, q_norm_w=
         if w is not None:
             _need(w, torch.bfloat16, name, 1)
     if q_out is None:
-        q_out = torch.empty(B, K, Hq, d, dtype=torch.bfloat16, device=qkv.device)
-    else:
-        _need(q_out, torch.bfloat16, "q_out", 4)
+        with _on(stream):
+            q_out = torch.empty(B, K, Hq, d, dtype=torch.bfloat16, device=qkv.device)
+    _need(q_out, torch.bfloat16, "q_out", 4)
     if dev_status is not None:
         _need(dev_status, torch.int32, "dev_status")
     rc = load().orthrus_block_qkv_append(_ptr(qkv), _ptr(q_norm_w), _ptr(k_norm_w),
