@@ -505,7 +505,7 @@ def run_ours(args):
                    "frac_of_bf16_peak": round(lm_tflops / tc_sus, 4),
                    "frac_of_bf16_peak_burst": round(lm_tflops / tc_peak, 4)},
         "roofline": {
-            "kernel": "orthrus_block_attn (cooperative split-KV kernel with in-kernel LSE merge), "
+            "kernel": "orthrus_block_attn (persistent split-KV kernel with in-kernel LSE merge), "
                       "AR and DIFF masks",
             "bound": "hbm",
             "achieved": round(attn_gbs, 1),

@@ -152,10 +152,15 @@ int orthrus_block_attn_workspace_size(int B, int Hq, int Hkv, int d, int K, size
  *   dev_status int32 device or NULL (see conventions; ORTHRUS_ECAPACITY when
  *              L_b + K > cap, in which case L_b is clamped to cap - K)
  * Supported: d in {64, 128}; 1 <= K <= 32; Hq / Hkv <= 128.
- * Runs as one cooperative, persistent split-KV kernel (one CTA per SM, tcgen05
- * MMAs with TMEM accumulators, TMA-staged K/V tiles) whose CTAs merge their
- * partial results by log-sum-exp: per segment, behind that segment's counter,
- * when every segment gets its own CTAs; after a grid barrier otherwise.
+ * Runs as one persistent split-KV kernel (one CTA per SM, tcgen05 MMAs with
+ * TMEM accumulators, TMA-staged K/V tiles) whose CTAs merge their partial
+ * results by log-sum-exp: per segment, behind that segment's counter, when
+ * every segment gets its own CTAs; after a grid barrier otherwise.  Every CTA
+ * must be resident at once.  With programmatic dependent launch on (the
+ * default) the launch is plain, so back-to-back calls overlap; work that other
+ * streams run at the same time can then hold SMs some CTAs wait for (past the
+ * wait limit: ORTHRUS_ETIMEOUT).  Setting ORTHRUS_ATTN_COOPERATIVE (or
+ * ORTHRUS_NO_PDL) before the first call makes every launch cooperative.
  */
 int orthrus_block_attn(const void *q, const orthrus_kv_cache *cache, int Hq, int K,
                        int mask_mode, void *out, void *workspace, size_t ws_bytes,
