@@ -69,8 +69,9 @@ constexpr int TN = 64;        // keys per compute tile
 // 80% of it, 128-row boxes near 97%).
 constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
 // Load groups of its static run a CTA asks L2 to prefetch while it still waits
-// for the previous kernel in the stream (4 groups = 256 KB of K and V at D = 128).
-constexpr int PREFETCH_GROUPS = 4;
+// for the previous kernel in the stream (2 groups = 128 KB of K and V at D = 128;
+// measured in the decode step: 2 beat 0 and 4).
+constexpr int PREFETCH_GROUPS = 2;
 // Partial O layout: [ROWS / BR row blocks][slot][D / 4 column quads][BR rows][4]
 // floats.  A warp's store of one column quad for its 32 rows covers four whole
 // 128-byte lines, and since the pieces of a segment occupy consecutive slots,
@@ -1005,9 +1006,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   // guess costs bandwidth, never a result; the schedule itself is computed
   // again after the wait.  Rows past the cache view are dropped by the tensor
   // map's bounds.
+  int raw_pre = 0;        // lane b: ctx_lens[b] as read before the wait
+  bool have_pre = false;  // the schedule in shared memory was computed from raw_pre
   if (warp == 0 && p.B <= 32 && p.balance) {
-    warp_schedule_small(p, gridDim.x, blockIdx.x, lane, false, sched,
-                        lane < p.B ? __ldcg(p.ctx_lens + lane) : 0);
+    raw_pre = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
+    warp_schedule_small(p, gridDim.x, blockIdx.x, lane, false, sched, raw_pre);
+    have_pre = true;
     __syncwarp();
     if (lane == 0) {
       const OwnSeg g0 = read_own();
@@ -1031,7 +1035,19 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   grid_dep_wait();
   if (warp == 0) {
-    warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
+    if (have_pre) {
+      // The schedule is a function of the lengths alone: if every length reads
+      // as it did before the wait, the one already in shared memory stands.
+      const int raw = lane < p.B ? __ldcg(p.ctx_lens + lane) : 0;
+      if (__all_sync(0xFFFFFFFFu, raw == raw_pre)) {
+        if (blockIdx.x == 0 && lane < p.B && (raw < 0 || raw > p.cap - p.K))
+          report(p.dev_status, ORTHRUS_ECAPACITY);
+      } else {
+        warp_schedule_small(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched, raw);
+      }
+    } else {
+      warp_schedule(p, gridDim.x, blockIdx.x, lane, blockIdx.x == 0, sched);
+    }
     __syncwarp();
   }
   // warps 0 and 1 meet: the barriers are initialised and the schedule written
@@ -1473,9 +1489,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row1e = BR * static_cast<int>(mul_div(k + 1, nblk, own.cn));
     const int row1 = row1e < RV ? row1e : RV;
     if (threadIdx.x == 0) {
-      fence_acq_rel_gpu();  // release this CTA's partial (written before the CTA barrier)
+      // the release covers this CTA's partial (written before the CTA barrier)
       const unsigned long long add = k == 0 ? (1ull << 20) - (own.cn - 1) : 1ull;
-      const unsigned long long old = atomicAdd(p.seg_cnt + own.s, add);
+      const unsigned long long old = atom_add_release_gpu(p.seg_cnt + own.s, add);
       if (row1 > row0 &&
           grid_wait(p.seg_cnt + own.s, ((old >> 20) + 1) << 20, p.dev_status, p.wait_ns) &&
           k == own.cn - 1 && p.balance)

@@ -166,6 +166,16 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 }
 // Acquire load at gpu scope: later reads of this thread observe every write
 // released before the value it returns was written.
+// Atomic add with release semantics at GPU scope (the thread's earlier writes,
+// and those ordered before it by a CTA barrier, are visible to whoever
+// acquires the new value); returns the old value.
+__device__ __forceinline__ unsigned long long atom_add_release_gpu(unsigned long long* a,
+                                                                 unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.release.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(a), "l"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ unsigned long long ld_acquire_gpu(const unsigned long long* p) {
   unsigned long long v;
   asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
