@@ -72,6 +72,12 @@ constexpr int ROWS = 128;     // query rows per tile (tcgen05 M)
 // for the previous kernel in the stream (2 groups = 128 KB of K and V at D = 128;
 // measured in the decode step: 2 beat 0 and 4).
 constexpr int PREFETCH_GROUPS = 2;
+// Balanced mode: the claim pool's last TAIL_HALF_GROUPS * cn / 2 groups (cn =
+// the segment's CTAs) are handed out as single 64-key tiles.  Measured in the
+// decode step (40960 x K 32): 0, i.e. whole groups to the end, is fastest; a
+// lone tile costs a ring item, an S sequence and a softmax pass for half the
+// keys, more than the tighter finish it buys (1 cost 0.4 us, 2 cost 0.9 us).
+constexpr int TAIL_HALF_GROUPS = 0;
 // Partial O layout: [ROWS / BR row blocks][slot][D / 4 column quads][BR rows][4]
 // floats.  A warp's store of one column quad for its 32 rows covers four whole
 // 128-byte lines, and since the pieces of a segment occupy consecutive slots,
@@ -882,10 +888,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     pr_pend = atomicAdd(p.seg_next + pr_own.s, 1ull);
     pr_grabbing = true;
   };
-  // Work units are (first tile << 1) | pair.  The static run and the pool's
-  // first claims are 128-key groups; the pool's last groups (one per sibling)
-  // are handed out as single 64-key tiles, which halves the spread of the
-  // siblings' finishing times.
+  // Work units are (first tile << 1) | pair.  The static run and the claims
+  // are 128-key groups (the pool's last TAIL_HALF_GROUPS * cn / 2 groups, if
+  // any, as single 64-key tiles).
   auto group_unit = [&](int g) { return (4 * g) | (2 * g + 1 < pr_own.ns ? 1 : 0); };
   auto next_unit = [&]() -> int {
     if (pr_sg < pr_sg_end) {
@@ -1065,7 +1070,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       pr_sg_end = pr_sg + fs;
       pr_dry = pr_pool0 >= pr_ngr;
       const int pool = pr_ngr - pr_pool0;             // groups left to claim
-      pr_gclaims = pool > pr_own.cn ? pool - pr_own.cn : 0;
+      const int tail = (TAIL_HALF_GROUPS * pr_own.cn + 1) / 2;  // groups cut into tiles
+      pr_gclaims = pool > tail ? pool - tail : 0;
       pr_tile0 = 2 * (pr_pool0 + pr_gclaims);         // then tiles from here
     }
     produce(NK, true);
