@@ -78,6 +78,9 @@ constexpr int PREFETCH_GROUPS = 2;
 // lone tile costs a ring item, an S sequence and a softmax pass for half the
 // keys, more than the tighter finish it buys (1 cost 0.4 us, 2 cost 0.9 us).
 constexpr int TAIL_HALF_GROUPS = 0;
+// Balanced mode: each CTA first streams a static run of STATIC_NUM / STATIC_DEN
+// of its fair share of the segment's groups, then claims.
+constexpr int STATIC_NUM = 3, STATIC_DEN = 4;
 // Partial O layout: [ROWS / BR row blocks][slot][D / 4 column quads][BR rows][4]
 // floats.  A warp's store of one column quad for its 32 rows covers four whole
 // 128-byte lines, and since the pieces of a segment occupy consecutive slots,
@@ -1022,7 +1025,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const OwnSeg g0 = read_own();
       if (g0.s >= 0 && g0.cn > 0) {
         const int k = static_cast<int>(blockIdx.x) - g0.c0;
-        const int fs = static_cast<int>(mul_div(3 * ((g0.ns + 1) / 2), 1, 4 * g0.cn));
+        const int fs = static_cast<int>(
+            mul_div(STATIC_NUM * ((g0.ns + 1) / 2), 1, STATIC_DEN * g0.cn));
         const int b = static_cast<int>(g0.s) / nseg, seg = static_cast<int>(g0.s) - b * nseg;
         const int kvbase = (b * p.Hkv + seg / p.nhc) * p.cap;
         const int n = fs < PREFETCH_GROUPS ? fs : PREFETCH_GROUPS;
@@ -1064,7 +1068,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (pr_own.s >= 0 && p.balance) {
       const int k = static_cast<int>(blockIdx.x) - pr_own.c0;
       pr_ngr = (pr_own.ns + 1) / 2;
-      const int fs = static_cast<int>(mul_div(3 * pr_ngr, 1, 4 * pr_own.cn));
+      const int fs = static_cast<int>(mul_div(STATIC_NUM * pr_ngr, 1, STATIC_DEN * pr_own.cn));
       pr_pool0 = pr_own.cn * fs;
       pr_sg = k * fs;
       pr_sg_end = pr_sg + fs;
