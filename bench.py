@@ -16,8 +16,9 @@ the launching stream inside the timed region.
 
 On one GPU the line also carries, unless --no-extras: the ragged-batch step (8
 sequences, lengths U[1024, 32768], K 32, planted accept lengths U{0..32}; its
-LM head has R = 256 rows) and the verify-step sweep over K in {1,4,8,16,32} x
-context in {1024, 8192, 40960, 131072} (K = 1 is plain decoding).
+LM head has R = 256 rows, timed in the step and alone) and the verify-step
+sweep over K in {1,4,8,16,32} x context in {1024, 8192, 40960, 131072} (K = 1
+is plain decoding).
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload (the reference arm of this benchmark).  Under torchrun (N > 1) every
@@ -695,9 +696,37 @@ def run_ragged(dev, stream, hbm_peak, tc_peak, tc_sus, n_steps=8):
                         "GB_per_s": round(wl.lm_bytes() / (lm_us * 1e-6) / 1e9, 1)},
         "device_status": int(wl.status.item()),
     }
+    out["lmhead_r256_alone"] = time_lmhead_alone(wl, stream, tc_peak)
     del wl
     torch.cuda.empty_cache()
     return out
+
+
+def time_lmhead_alone(wl, stream, tc_peak, launches=10):
+    """The step's AR-pass LM head (same h, W and workspace) timed alone: a CUDA
+    graph of back-to-back launches, timed after one warm replay.  W (1.2 GB) is
+    larger than L2, so every launch streams it from HBM; a kernel timed alone
+    takes the burst bf16 peak."""
+    import torch
+    from lossless_block_drafting_b200 import orthrus as ob
+    with torch.cuda.stream(stream):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for _ in range(launches):
+                ob.lmhead_argmax(wl.h_ar, wl.W, argmax=wl.argmax, workspace=wl.ws_lm,
+                                 stream=stream, dev_status=wl.status)
+        gr.replay()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        gr.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / launches
+    tf = wl.lm_flops() / (us * 1e-6) / 1e12
+    del gr
+    return {"us_per_call": round(us, 2), "TFLOP_per_s": round(tf, 1),
+            "frac_of_bf16_peak_burst": round(tf / tc_peak, 4), "launches": launches,
+            "device_status": int(wl.status.item())}
 
 
 def run_step_with_append(dev, stream, L, K, layers, accept, n_steps=8):
